@@ -1,0 +1,116 @@
+"""Seeded synthetic inputs and the named workloads.
+
+This module generates inputs only; it holds none of the attention arithmetic.
+Both the GPU path's tests/benchmark and the CPU oracle take their inputs from
+here, so that both sides see identical bf16 (or fp16) values.
+
+Recipe: a CPU ``torch.Generator`` seeded with ``seed`` draws fp32 standard
+normals for Q, K and V in that order; the workload's transforms are applied in
+fp32 (a uniform multiplier; for the outlier recipe, an independent
+Bernoulli(p) mask per element, drawn after the normals, that multiplies the
+chosen entries by a factor); the result is rounded to the storage dtype with
+round-to-nearest-even (torch's conversion).
+
+Workload shapes follow the pages' measurement set-up ("从理论到实现…" §6.1:
+d_model = 512 with 16 heads, sequence lengths 1024 and 16384) and the head
+dimension / length grid of the FlashAttention IO analysis on the "Flash
+Attention" tag page (n = 8192, d = 128).
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+
+@dataclass(frozen=True)
+class Case:
+    """One attention problem: shape, mask, value recipe and seed."""
+
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    causal: bool
+    seed: int
+    value_scale: float = 1.0
+    outlier_frac: float = 0.0
+    outlier_mult: float = 8.0
+    fp8: bool = False
+
+    @property
+    def softmax_scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def flops(self) -> float:
+        f = 4.0 * self.B * self.H * float(self.N) ** 2 * self.d
+        return f / 2 if self.causal else f
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    cases: tuple = field(default_factory=tuple)
+    description: str = ""
+
+
+def _c(name, B, H, N, d, causal, seed, **kw):
+    return Case(name, B, H, N, d, causal, seed, **kw)
+
+
+WORKLOADS = {
+    "tiny": Workload("tiny", (
+        _c("tiny_b1h2n256d64", 1, 2, 256, 64, False, 0),),
+        "B=1 H=2 N=256 d=64 non-causal, N(0,1)"),
+    "dmodel512_h16": Workload("dmodel512_h16", (
+        _c("b1h16n1024d32_causal", 1, 16, 1024, 32, True, 1),
+        _c("b1h16n1024d32", 1, 16, 1024, 32, False, 1),
+        _c("b1h16n16384d32_causal", 1, 16, 16384, 32, True, 1),
+        _c("b1h16n16384d32", 1, 16, 16384, 32, False, 1),),
+        "d_model=512 with 16 heads: B=1 H=16 d=32, N in {1024, 16384}, causal and non-causal, N(0,1)"),
+    "b4h16n8192d128_causal": Workload("b4h16n8192d128_causal", (
+        _c("b4h16n8192d128_causal", 4, 16, 8192, 128, True, 2, value_scale=0.5),),
+        "B=4 H=16 N=8192 d=128 causal, N(0,1)*0.5, LSE written"),
+    "b1h32n32768d128_causal": Workload("b1h32n32768d128_causal", (
+        _c("b1h32n32768d128_causal", 1, 32, 32768, 128, True, 3),),
+        "B=1 H=32 N=32768 d=128 causal, N(0,1)"),
+    "fp8_b2h16n16384d128_causal": Workload("fp8_b2h16n16384d128_causal", (
+        _c("fp8_b2h16n16384d128_causal", 2, 16, 16384, 128, True, 4,
+           outlier_frac=0.01, outlier_mult=8.0, fp8=True),),
+        "FP8 e4m3 Q/K with per-128-row-tile scales, V bf16: B=2 H=16 N=16384 d=128 causal, "
+        "N(0,1) with 1% of entries x8"),
+    # non-causal d=128 long-sequence cases (the throughput target's shape)
+    "target_d128_noncausal": Workload("target_d128_noncausal", (
+        _c("b4h16n8192d128", 4, 16, 8192, 128, False, 2, value_scale=0.5),
+        _c("b1h32n16384d128", 1, 32, 16384, 128, False, 5),),
+        "B=4 H=16 N=8192 d=128 and B=1 H=32 N=16384 d=128, non-causal"),
+}
+
+
+def make_qkv(case: Case, dtype=torch.bfloat16, device="cpu"):
+    """Seeded Q, K, V of ``case``'s shape, rounded to ``dtype`` (RNE)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(case.seed)
+    shape = (case.B, case.H, case.N, case.d)
+    out = []
+    raw = [torch.randn(shape, generator=g, dtype=torch.float32) for _ in range(3)]
+    if case.outlier_frac > 0:
+        for t in raw:
+            mask = torch.rand(shape, generator=g, dtype=torch.float32) < case.outlier_frac
+            t[mask] *= case.outlier_mult
+    for t in raw:
+        if case.value_scale != 1.0:
+            t *= case.value_scale
+        out.append(t.to(dtype).to(device))
+    return tuple(out)
+
+
+def make_tensor(shape, seed: int, dtype=torch.bfloat16, scale: float = 1.0):
+    """A single seeded N(0,1)*scale tensor (for edge-case tests)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    return (torch.randn(shape, generator=g, dtype=torch.float32) * scale).to(dtype)
