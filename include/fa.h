@@ -1,0 +1,139 @@
+/*
+ * fa.h — C ABI of the B200 (sm_100a) FlashAttention forward library.
+ *
+ * The operation (every entry point below computes a part of it):
+ *
+ *     S   = softmax_scale * Q K^T                 per (batch, head)
+ *     S[i,j] = -inf  where causal and j > i       (top-left aligned)
+ *     O   = softmax(S) V                          row-wise softmax
+ *     LSE[i] = log(sum_j exp(S[i,j]))             natural log
+ *
+ * Definition: the "Flash Attention" tag page (guijiagi.com), excerpt "Flash
+ * Attention解决了什么问题", section 算法原理 (S = QK^T/sqrt(d), P = softmax(S),
+ * O = PV), with the (batch, heads, seq, dim) layout of the excerpt "Flash
+ * Attention 系列回顾".  The tile-by-tile online-softmax evaluation follows
+ * "从理论到实现：基于Triton剖析FlashAttention三代的演进与优化" §2.1; the block
+ * causal mask follows §3.1 of the same article; the FP8 path with dynamic
+ * per-tile scales folded into the score scale follows its §4.1.  The caller-set
+ * softmax scale is the FlashAttention(softmax_scale=...) argument of
+ * "FlashAttention速度提升的核心原理" §4.2.
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors are dense, contiguous, row-major [B, H, N, d] (d fastest) in
+ *     device memory owned by the caller.  Base pointers must be 16-byte
+ *     aligned.  LSE is fp32 [B, H, N].
+ *   - d (head dimension) is 32, 64 or 128.  Any N >= 1 is accepted; the ragged
+ *     tail is handled inside the kernels.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t, passed as void*;
+ *     NULL means the legacy default stream).  They do not synchronise the host.
+ *   - Arguments are validated before any CUDA call; invalid arguments return
+ *     FA_ERR_INVALID / FA_ERR_UNSUPPORTED and touch no device state.
+ *   - Kernels never trap.  Every wait inside a kernel is bounded; a wait that
+ *     runs out sets a device status word (read by fa_last_device_status) and
+ *     the kernel exits cleanly.
+ *   - Not thread-safe against concurrent calls that grow the FA_E4M3
+ *     workspace of the same device; all other calls may be issued from any
+ *     thread.
+ */
+#ifndef FA_SM100_H_
+#define FA_SM100_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID = 1,      /* null pointer, bad size, misalignment, bad scale  */
+  FA_ERR_UNSUPPORTED = 2,  /* head dimension or dtype this build does not have */
+  FA_ERR_ARCH = 3,         /* current device is not compute capability 10.x    */
+  FA_ERR_CUDA = 4,         /* a CUDA runtime/driver call or launch failed      */
+  FA_ERR_TIMEOUT = 5       /* a kernel gave up on a bounded wait               */
+} fa_status;
+
+typedef enum {
+  FA_BF16 = 0,   /* Q, K, V, O bf16; P rounded to bf16 for the P V product     */
+  FA_FP16 = 1,   /* Q, K, V, O fp16; P rounded to fp16                         */
+  FA_E4M3 = 2    /* Q, K given as bf16 and quantised by the library to e4m3
+                    with one scale per (batch, head, 128-row tile); V, O bf16   */
+} fa_dtype;
+
+/*
+ * fa_fwd — the forward pass.
+ *   q, k, v : [B, H, N, d] inputs (bf16 / fp16 per dtype; for FA_E4M3, bf16).
+ *   o       : [B, H, N, d] output, same element type as v.  Must not alias
+ *             q, k or v.
+ *   lse     : [B, H, N] fp32 output, or NULL to skip writing it.
+ *   softmax_scale : finite, > 0 (typically 1/sqrt(d)).
+ *   causal  : 0 or 1.
+ * For FA_E4M3 the library quantises q and k into a workspace it owns (grown
+ * on demand with cudaMalloc, freed by fa_release) and then runs the FP8
+ * attention kernel; this path therefore allocates on first use or growth.
+ * Returns FA_OK once the work is enqueued.
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int H, int N, int d, float softmax_scale, int causal,
+                 fa_dtype dtype, void* stream);
+
+/*
+ * fa_quantize_e4m3 — per-tile dynamic-scale quantiser ("从理论到实现…" §4.1,
+ * with the e4m3 constant 448 in place of int8's 127).
+ *   x      : [B, H, N, d] bf16 input.
+ *   x8     : [B, H, N, d] uint8 output, e4m3 codes (RNE, saturating).
+ *   scales : [B, H, ceil(N/128)] fp32 output; scale = 448 / amax over the
+ *            tile's rows x d, or 1 for an all-zero tile.  code = e4m3(x*scale).
+ */
+fa_status fa_quantize_e4m3(const void* x, void* x8, float* scales,
+                           int B, int H, int N, int d, void* stream);
+
+/*
+ * fa_fwd_fp8 — attention on pre-quantised Q and K.
+ *   q8, k8   : [B, H, N, d] e4m3 codes; q_scale, k_scale : [B, H, ceil(N/128)]
+ *              fp32 scales as written by fa_quantize_e4m3.  The kernel uses
+ *              S = softmax_scale * (q8 . k8) / (q_scale[tile(i)] * k_scale[tile(j)]).
+ *   v, o     : bf16 [B, H, N, d];  lse as in fa_fwd.  d must be 128.
+ */
+fa_status fa_fwd_fp8(const void* q8, const float* q_scale, const void* k8, const float* k_scale,
+                     const void* v, void* o, float* lse, int B, int H, int N, int d,
+                     float softmax_scale, int causal, void* stream);
+
+/*
+ * fa_last_device_status — synchronises `stream`, reads and clears the device
+ * status word of the current device.  FA_OK when no kernel on this device
+ * gave up on a wait since the last call; FA_ERR_TIMEOUT otherwise.
+ */
+fa_status fa_last_device_status(void* stream);
+
+/* fa_status_string — static, never-NULL description of a status code. */
+const char* fa_status_string(fa_status status);
+
+/*
+ * fa_release — frees library-owned device memory (the FA_E4M3 workspace and
+ * the status word) of the current device.  Call only with no library work in
+ * flight on that device.
+ */
+fa_status fa_release(void);
+
+/*
+ * fa_debug_set_wait_limit — test hook.  Sets the bound, in nanoseconds, that
+ * every in-kernel wait uses before giving up (0 restores the default of
+ * 2 seconds).  Lets a test make a wait run out without hanging the GPU.
+ */
+fa_status fa_debug_set_wait_limit(uint64_t nanoseconds);
+
+/*
+ * fa_debug_withhold_arrival — test hook.  When nonzero, the next fa_fwd
+ * launch runs with the load warp skipping its first K/V tile load, so the
+ * consumers' bounded waits run out and the kernel reports FA_ERR_TIMEOUT.
+ * Cleared after one launch.
+ */
+fa_status fa_debug_withhold_arrival(int enable);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_SM100_H_ */

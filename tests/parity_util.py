@@ -1,0 +1,51 @@
+"""Shared helpers for the GPU parity tests: tolerance gates and row samples."""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+# Tolerances (max-abs, mean-abs, LSE abs) for 16-bit and FP8 paths.
+TOL_16 = (1e-2, 1e-3, 1e-3)
+TOL_FP8 = (6e-2, 1e-3, 1e-3)
+
+
+def half_ulp(ref: np.ndarray, dtype) -> np.ndarray:
+    """Half a unit in the last place of the output format at |ref|: the error
+    that rounding a perfect fp32 result to the stored 16-bit type can add."""
+    mant = 7 if dtype == torch.bfloat16 else 10
+    min_exp = -126 if dtype == torch.bfloat16 else -14
+    a = np.maximum(np.abs(ref), 2.0 ** min_exp)
+    e = np.floor(np.log2(a))
+    return 2.0 ** (e - mant) / 2
+
+
+def gate(o_gpu, o_ref, lse_gpu=None, lse_ref=None, tol=TOL_16, out_dtype=torch.bfloat16, what=""):
+    """Element-wise parity: max over elements of (|o - ref| - half_ulp(ref)) and
+    the raw mean-abs error, plus the raw LSE error.  Returns the measured errors."""
+    o = o_gpu.detach().float().cpu().double().numpy() if hasattr(o_gpu, "detach") else np.asarray(o_gpu)
+    err = np.abs(o - o_ref)
+    excess = np.maximum(0.0, err - half_ulp(o_ref, out_dtype))
+    res = {"max_abs": float(err.max()), "max_excess": float(excess.max()), "mean_abs": float(err.mean())}
+    assert np.all(np.isfinite(o)), f"{what}: non-finite output"
+    assert res["max_excess"] <= tol[0], f"{what}: max excess {res}"
+    assert res["mean_abs"] <= tol[1], f"{what}: mean abs {res}"
+    if lse_ref is not None:
+        lg = lse_gpu.detach().double().cpu().numpy() if hasattr(lse_gpu, "detach") else np.asarray(lse_gpu)
+        le = np.abs(lg - lse_ref)
+        res["lse_max_abs"] = float(le.max())
+        assert res["lse_max_abs"] <= tol[2], f"{what}: lse {res}"
+    return res
+
+
+def sample_rows(N: int, seed: int, n_random: int = 96) -> np.ndarray:
+    """Rows at the start, around every kind of tile boundary, at the end, and
+    a seeded random spread."""
+    rng = np.random.default_rng(seed)
+    rows = set(range(min(N, 40)))
+    for b in (127, 128, 129, 255, 256, 257, 383, 384, 511, 512):
+        if b < N:
+            rows.add(b)
+    rows.update(range(max(0, N - 40), N))
+    rows.update(rng.integers(0, N, size=min(n_random, N)).tolist())
+    return np.array(sorted(rows), dtype=np.int64)

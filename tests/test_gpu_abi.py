@@ -1,0 +1,47 @@
+"""C ABI behaviour on the GPU: status codes, the bounded-wait timeout path."""
+
+from __future__ import annotations
+
+import pytest
+import torch
+
+import tiled_attention_12_b200 as fa
+from tiled_attention_12_b200 import binding as B
+from tiled_attention_12_b200.synth import Case, make_qkv
+
+pytestmark = pytest.mark.gpu
+
+
+def test_timeout_is_reported_and_context_survives():
+    """A K/V tile that never arrives: every wait gives up after the limit, the
+    kernel exits, the status word says so, and the next call works."""
+    c = Case("t", 1, 2, 512, 64, False, seed=5)
+    q, k, v = (t.cuda() for t in make_qkv(c))
+    assert fa.fa_last_device_status() == B.FA_OK
+    fa.fa_debug_set_wait_limit(20_000_000)       # 20 ms
+    fa.fa_debug_withhold_arrival(True)
+    try:
+        fa.fa_fwd(q, k, v)
+        assert fa.fa_last_device_status() == B.FA_ERR_TIMEOUT
+    finally:
+        fa.fa_debug_set_wait_limit(0)
+        fa.fa_debug_withhold_arrival(False)
+    o, _ = fa.fa_fwd(q, k, v)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status() == B.FA_OK
+    ref = torch.nn.functional.scaled_dot_product_attention(q.float(), k.float(), v.float())
+    assert (o.float() - ref).abs().max().item() < 2e-2
+
+
+def test_invalid_arguments_on_gpu():
+    c = Case("t", 1, 1, 64, 64, False, seed=6)
+    q, k, v = (t.cuda() for t in make_qkv(c))
+    L = B.load()
+    o = torch.empty_like(v)
+    s = torch.cuda.current_stream().cuda_stream
+    assert L.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), None, 1, 1, 64, 64, -1.0, 0, 0, s) == 1
+    assert L.fa_fwd(q.data_ptr() + 2, k.data_ptr(), v.data_ptr(), o.data_ptr(), None, 1, 1, 64, 64, 0.1, 0, 0, s) == 1
+    assert L.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), q.data_ptr(), None, 1, 1, 64, 64, 0.1, 0, 0, s) == 1
+    assert L.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), None, 1, 1, 64, 96, 0.1, 0, 0, s) == 2
+    assert L.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), None, 1, 1, 64, 64, 0.1, 0, 2, s) == 2
+    assert fa.fa_last_device_status() == B.FA_OK

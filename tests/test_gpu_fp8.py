@@ -1,0 +1,71 @@
+"""GPU parity of the e4m3 path: quantiser bit-exact, attention vs the oracle."""
+
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import tiled_attention_12_b200 as fa
+from oracle import (attention_ref, attention_rows, dequantize_e4m3_tiles, quantize_e4m3_tiles)
+from tiled_attention_12_b200.synth import WORKLOADS, Case, make_qkv
+
+from parity_util import TOL_FP8, gate, sample_rows
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+C5 = WORKLOADS["fp8_b2h16n16384d128_causal"].cases[0]
+
+
+@pytest.mark.parametrize("N,d", [(1, 128), (100, 128), (128, 64), (300, 32), (1000, 128)])
+def test_quantiser_bit_exact(N, d):
+    c = dataclasses.replace(C5, B=2, H=3, N=N, d=d)
+    q, _, _ = make_qkv(c)
+    q[0, 1, : min(N, 128)] = 0                     # an all-zero tile
+    codes, scales = fa.fa_quantize_e4m3(q.to(DEV))
+    torch.cuda.synchronize()
+    rc, rs = quantize_e4m3_tiles(q)
+    assert np.array_equal(scales.cpu().numpy(), rs)
+    assert np.array_equal(codes.cpu().numpy(), rc)
+
+
+def _fp8_case(c: Case, full: bool):
+    q, k, v = make_qkv(c)
+    o, lse = fa.fa_fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=c.causal, dtype=fa.FA_E4M3)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status() == 0
+    cq, sq = quantize_e4m3_tiles(q)
+    ck, sk = quantize_e4m3_tiles(k)
+    qd, kd = dequantize_e4m3_tiles(cq, sq), dequantize_e4m3_tiles(ck, sk)
+    if full:
+        o_ref, lse_ref = attention_ref(qd, kd, v, c.softmax_scale, c.causal)
+        gate(o, o_ref, lse, lse_ref, tol=TOL_FP8, what=c.name)
+        return
+    for b, h in sorted({(0, 0), (c.B - 1, c.H - 1), (c.B // 2, c.H // 2)}):
+        rows = sample_rows(c.N, seed=b * 100 + h)
+        o_ref, lse_ref = attention_rows(qd, kd, v, c.softmax_scale, c.causal, b, h, rows)
+        gate(o.cpu()[b, h][rows], o_ref, lse.cpu()[b, h][rows], lse_ref, tol=TOL_FP8, what=f"{c.name} {b},{h}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 129, 256, 700])
+def test_fp8_small(N, causal):
+    c = dataclasses.replace(C5, B=1, H=2, N=N, causal=causal)
+    _fp8_case(c, full=True)
+
+
+def test_fp8_named_workload():
+    _fp8_case(C5, full=False)
+
+
+def test_fp8_prequantised_entry_matches():
+    c = dataclasses.replace(C5, B=1, H=3, N=1000)
+    q, k, v = (t.to(DEV) for t in make_qkv(c))
+    o1, l1 = fa.fa_fwd(q, k, v, causal=True, dtype=fa.FA_E4M3)
+    q8, qs = fa.fa_quantize_e4m3(q)
+    k8, ks = fa.fa_quantize_e4m3(k)
+    o2, l2 = fa.fa_fwd_fp8(q8, qs, k8, ks, v, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)

@@ -1,0 +1,163 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle."""
+
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import tiled_attention_12_b200 as fa
+from oracle import attention_ref, attention_rows
+from tiled_attention_12_b200.synth import WORKLOADS, Case, make_qkv, make_tensor
+
+from parity_util import TOL_16, gate, sample_rows
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def run(q, k, v, causal, scale=None, dtype=None):
+    o, lse = fa.fa_fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=causal, softmax_scale=scale, dtype=dtype)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status() == fa.binding.FA_OK
+    return o, lse
+
+
+SMALL = [(1, 1, n, d) for n in (1, 7, 64, 128, 129, 255, 256, 257, 300, 640, 1000) for d in (32, 64, 128)]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", SMALL, ids=lambda s: "x".join(map(str, s)))
+def test_small_shapes_bf16(shape, causal):
+    B, H, N, d = shape
+    c = Case("s", B, H, N, d, causal, seed=N * 7 + d)
+    q, k, v = make_qkv(c)
+    o, lse = run(q, k, v, causal)
+    o_ref, lse_ref = attention_ref(q, k, v, c.softmax_scale, causal)
+    gate(o, o_ref, lse, lse_ref, what=f"{shape} causal={causal}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [32, 64, 128])
+def test_fp16_inputs(d, causal):
+    c = Case("f", 2, 3, 333, d, causal, seed=11 + d)
+    q, k, v = make_qkv(c, dtype=torch.float16)
+    o, lse = run(q, k, v, causal)
+    assert o.dtype == torch.float16
+    o_ref, lse_ref = attention_ref(q, k, v, c.softmax_scale, causal)
+    gate(o, o_ref, lse, lse_ref, out_dtype=torch.float16, what=f"fp16 d={d}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_many_work_tiles_persistent_loop(causal):
+    """More work tiles than SMs, ragged N: every CTA loops several times."""
+    c = Case("p", 3, 50, 700, 64, causal, seed=21)
+    q, k, v = make_qkv(c)
+    o, lse = run(q, k, v, causal)
+    o_ref, lse_ref = attention_ref(q, k, v, c.softmax_scale, causal)
+    gate(o, o_ref, lse, lse_ref, what="persistent")
+
+
+def test_lse_optional_and_custom_scale():
+    c = Case("n", 1, 4, 500, 128, True, seed=31)
+    q, k, v = make_qkv(c)
+    o, lse = fa.fa_fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=True, softmax_scale=0.37, want_lse=False)
+    torch.cuda.synchronize()
+    assert lse is None
+    o_ref, _ = attention_ref(q, k, v, 0.37, True)
+    gate(o, o_ref, what="no lse")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_invariant_rows_sum_to_one(causal):
+    c = Case("r", 1, 2, 1111, 128, causal, seed=41)
+    q, k, v = make_qkv(c)
+    v[..., 0] = 1.0
+    o, _ = run(q, k, v, causal)
+    assert torch.all((o[..., 0].float() - 1.0).abs() <= 1e-2)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_invariant_identical_v_rows(causal):
+    c = Case("i", 1, 2, 520, 64, causal, seed=42)
+    q, k, _ = make_qkv(c)
+    row = make_tensor((64,), 43)
+    v = row.expand(1, 2, 520, 64).contiguous()
+    o, _ = run(q, k, v, causal)
+    assert torch.max((o.float().cpu() - row.float()).abs()) <= 1e-2
+
+
+def test_invariant_causal_row_zero_is_v0_and_lse():
+    c = Case("z", 2, 2, 300, 128, True, seed=44)
+    q, k, v = make_qkv(c)
+    o, lse = run(q, k, v, True)
+    assert torch.equal(o[:, :, 0].cpu(), v[:, :, 0])
+    s00 = c.softmax_scale * (q[:, :, 0].double() * k[:, :, 0].double()).sum(-1)
+    assert torch.max((lse[:, :, 0].double().cpu() - s00).abs()) <= 1e-3
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_closed_form_zero_q(causal):
+    c = Case("q0", 1, 1, 777, 32, causal, seed=45)
+    _, k, v = make_qkv(c)
+    q = torch.zeros_like(k)
+    o, lse = run(q, k, v, causal)
+    vf = v[0, 0].double().numpy()
+    if causal:
+        ref = np.cumsum(vf, axis=0) / np.arange(1, 778)[:, None]
+        lref = np.log(np.arange(1, 778))
+    else:
+        ref = np.broadcast_to(vf.mean(axis=0), vf.shape)
+        lref = np.full(777, math.log(777))
+    gate(o[0, 0], ref, lse[0, 0], lref, what="zero q")
+
+
+def test_large_scores_stay_finite():
+    c = Case("big", 1, 2, 400, 64, False, seed=46)
+    q, k, v = make_qkv(c)
+    q, k = (q.float() * 100).to(torch.bfloat16), (k.float() * 100).to(torch.bfloat16)
+    o, lse = run(q, k, v, False)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+    o_ref, lse_ref = attention_ref(q, k, v, c.softmax_scale, False)
+    # scores are ~1e3 here: an fp32 rounding of S moves them by ~1e-4 relative
+    gate(o, o_ref, lse, lse_ref, tol=(5e-2, 5e-3, 5e-2), what="x100")
+
+
+def test_single_key():
+    c = Case("one", 2, 3, 1, 128, False, seed=47)
+    q, k, v = make_qkv(c)
+    for causal in (False, True):
+        o, lse = run(q, k, v, causal)
+        assert torch.equal(o.cpu(), v)
+
+
+# ------------------------------------------------------------ named workloads
+
+
+def _full_or_sampled(case: Case, dtype=torch.bfloat16, max_full_flops=2e10):
+    q, k, v = make_qkv(case, dtype=dtype)
+    o, lse = run(q, k, v, case.causal)
+    if case.flops <= max_full_flops:
+        o_ref, lse_ref = attention_ref(q, k, v, case.softmax_scale, case.causal)
+        return gate(o, o_ref, lse, lse_ref, what=case.name)
+    heads = sorted({(0, 0), (case.B - 1, case.H - 1), (case.B // 2, case.H // 2)})
+    o_c, lse_c = o.cpu(), lse.cpu()
+    for b, h in heads:
+        rows = sample_rows(case.N, seed=b * 1000 + h)
+        o_ref, lse_ref = attention_rows(q, k, v, case.softmax_scale, case.causal, b, h, rows)
+        gate(o_c[b, h][rows], o_ref, lse_c[b, h][rows], lse_ref, what=f"{case.name} b{b} h{h}")
+    # a property that holds at any size: ones in V give ones in O, every row
+    v1 = v.clone()
+    v1[..., 0] = 1.0
+    o1, _ = run(q, k, v1, case.causal)
+    assert torch.all((o1[..., 0].float() - 1.0).abs() <= 1e-2), case.name
+
+
+@pytest.mark.parametrize("case", [c for w in ("tiny", "dmodel512_h16", "b4h16n8192d128_causal",
+                                              "b1h32n32768d128_causal", "target_d128_noncausal")
+                                  for c in WORKLOADS[w].cases], ids=lambda c: c.name)
+def test_named_workload(case):
+    _full_or_sampled(case)

@@ -1,0 +1,166 @@
+"""ctypes binding of the C ABI in include/fa.h (argument marshalling only).
+
+Each function takes torch tensors (or raw integers for pointers), checks the
+shapes and dtypes the C side cannot see, passes data pointers and the current
+CUDA stream, and raises :class:`FaError` on a non-OK status.  All computation
+happens in the CUDA library; there is no fallback path.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+from .build import INCLUDE, LIB
+
+FA_OK, FA_ERR_INVALID, FA_ERR_UNSUPPORTED, FA_ERR_ARCH, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(6)
+FA_BF16, FA_FP16, FA_E4M3 = 0, 1, 2
+
+_lib = None
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = load().fa_status_string(status).decode()
+        super().__init__(f"{where}: status {status} ({msg})")
+
+
+def declared_symbols() -> list[str]:
+    """Names of the functions include/fa.h declares."""
+    text = open(os.path.join(INCLUDE, "fa.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:fa_status|const char\*)\s+(fa_\w+)\s*\(", text, re.M)))
+
+
+def load():
+    """Loads the in-tree library; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB):
+        raise RuntimeError(f"CUDA library missing at {LIB}; build it with "
+                           "`python -m tiled_attention_12_b200.build`")
+    L = ctypes.CDLL(LIB)
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
+    L.fa_quantize_e4m3.argtypes = [vp, vp, vp, i, i, i, i, vp]
+    L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    L.fa_last_device_status.argtypes = [vp]
+    L.fa_status_string.argtypes = [i]
+    L.fa_status_string.restype = ctypes.c_char_p
+    L.fa_release.argtypes = []
+    L.fa_debug_set_wait_limit.argtypes = [ctypes.c_uint64]
+    L.fa_debug_withhold_arrival.argtypes = [i]
+    for name in ("fa_fwd", "fa_quantize_e4m3", "fa_fwd_fp8", "fa_last_device_status", "fa_release",
+                 "fa_debug_set_wait_limit", "fa_debug_withhold_arrival"):
+        getattr(L, name).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def _check(status: int, where: str):
+    if status != FA_OK:
+        raise FaError(status, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return t if isinstance(t, int) else t.data_ptr()
+
+
+def _stream(stream):
+    import torch
+
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def _dtype_code(t):
+    import torch
+
+    if t.dtype == torch.bfloat16:
+        return FA_BF16
+    if t.dtype == torch.float16:
+        return FA_FP16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def fa_fwd(q, k, v, o=None, lse=None, softmax_scale=None, causal=False, dtype=None, stream=None,
+           want_lse=True):
+    """Forward pass on [B, H, N, d] CUDA tensors.  Returns (o, lse).
+
+    dtype: None (from q: bf16 or fp16) or FA_E4M3 (q, k bf16, quantised by the
+    library).  Output tensors are allocated when not given.
+    """
+    import torch
+
+    for t in (q, k, v):
+        if not (t.is_cuda and t.is_contiguous() and t.dim() == 4):
+            raise ValueError("q, k, v must be contiguous 4-D CUDA tensors")
+    if q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v shapes differ")
+    B, H, N, d = q.shape
+    code = _dtype_code(q) if dtype is None else dtype
+    if o is None:
+        o = torch.empty_like(v)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
+    scale = (1.0 / d ** 0.5) if softmax_scale is None else float(softmax_scale)
+    st = load().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, scale,
+                       int(bool(causal)), code, _stream(stream))
+    _check(st, "fa_fwd")
+    return o, lse
+
+
+def fa_quantize_e4m3(x, x8=None, scales=None, stream=None):
+    """Per-(b, h, 128-row tile) e4m3 quantisation.  Returns (codes uint8, scales fp32)."""
+    import torch
+
+    B, H, N, d = x.shape
+    if x8 is None:
+        x8 = torch.empty((B, H, N, d), device=x.device, dtype=torch.uint8)
+    if scales is None:
+        scales = torch.empty((B, H, (N + 127) // 128), device=x.device, dtype=torch.float32)
+    st = load().fa_quantize_e4m3(_ptr(x), _ptr(x8), _ptr(scales), B, H, N, d, _stream(stream))
+    _check(st, "fa_quantize_e4m3")
+    return x8, scales
+
+
+def fa_fwd_fp8(q8, q_scale, k8, k_scale, v, o=None, lse=None, softmax_scale=None, causal=False,
+               stream=None, want_lse=True):
+    """Attention on pre-quantised e4m3 Q/K codes (uint8 tensors) with bf16 V."""
+    import torch
+
+    B, H, N, d = v.shape
+    if o is None:
+        o = torch.empty_like(v)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, N), device=v.device, dtype=torch.float32)
+    scale = (1.0 / d ** 0.5) if softmax_scale is None else float(softmax_scale)
+    st = load().fa_fwd_fp8(_ptr(q8), _ptr(q_scale), _ptr(k8), _ptr(k_scale), _ptr(v), _ptr(o), _ptr(lse),
+                           B, H, N, d, scale, int(bool(causal)), _stream(stream))
+    _check(st, "fa_fwd_fp8")
+    return o, lse
+
+
+def fa_last_device_status(stream=None) -> int:
+    return load().fa_last_device_status(_stream(stream))
+
+
+def fa_status_string(status: int) -> str:
+    return load().fa_status_string(status).decode()
+
+
+def fa_release() -> int:
+    return load().fa_release()
+
+
+def fa_debug_set_wait_limit(ns: int) -> int:
+    return load().fa_debug_set_wait_limit(ns)
+
+
+def fa_debug_withhold_arrival(enable: bool) -> int:
+    return load().fa_debug_withhold_arrival(int(enable))

@@ -1,0 +1,283 @@
+// fa_api.cu — the C ABI declared in include/fa.h: argument validation, TMA
+// tensor-map creation, per-device state, launches.
+//
+// Validation happens before any CUDA call, so bad arguments are reported
+// without touching the device.  Nothing here computes attention; every step
+// of the path runs in the kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_fwd_kernel.cuh"
+#include "fa_launch.h"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s
+
+struct DeviceState {
+  bool ready = false;
+  int sms = 0;
+  int major = 0;
+  unsigned int* status = nullptr;  // device status word
+  void* ws = nullptr;              // FA_E4M3 workspace
+  size_t ws_bytes = 0;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+EncodeTiledFn g_encode = nullptr;
+uint64_t g_wait_ns = kDefaultWaitNs;
+int g_withhold = 0;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fa_status map_cuda(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
+
+// Current device, its state (created on first use), checked to be sm_100.
+fa_status device_state(DeviceState** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& s = g_dev[dev];
+  if (!s.ready) {
+    int major = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return FA_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FA_ERR_CUDA;
+    s.major = major;
+    s.sms = sms;
+    if (major != 10) return FA_ERR_ARCH;
+    if (cudaMalloc(&s.status, sizeof(unsigned int)) != cudaSuccess) return FA_ERR_CUDA;
+    if (cudaMemset(s.status, 0, sizeof(unsigned int)) != cudaSuccess) return FA_ERR_CUDA;
+    if (g_encode == nullptr) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return FA_ERR_CUDA;
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    s.ready = true;
+  }
+  if (s.major != 10) return FA_ERR_ARCH;
+  *out = &s;
+  return FA_OK;
+}
+
+// [BH, N, d] tensor viewed as a 3-D TMA map {d, N, BH}; box {64 (or d) elements
+// of 16 bits | 128 bytes of 8 bits, 128 rows, 1 head}, swizzled to match the
+// tcgen05 shared-memory layout.
+fa_status make_map(CUtensorMap* map, const void* ptr, int BH, int N, int d, int elem_bytes, bool fp16) {
+  const CUtensorMapDataType dt = elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : (fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+  const int row_bytes = d * elem_bytes;
+  const int span = row_bytes >= 128 ? 128 : row_bytes;
+  const CUtensorMapSwizzle sw = span == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(row_bytes) * N};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(span / elem_bytes), 128u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = g_encode(map, dt, 3, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_INVALID;
+}
+
+fa_status check_shape(int B, int H, int N, int d) {
+  if (B <= 0 || H <= 0 || N <= 0) return FA_ERR_INVALID;
+  const long long bh = static_cast<long long>(B) * H;
+  const long long qpairs = (static_cast<long long>(N) + 255) / 256;
+  if (bh > 0x7FFFFFFFLL || bh * qpairs > 0x7FFFFFFFLL) return FA_ERR_INVALID;
+  if (d != 32 && d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+bool scale_ok(float s) { return std::isfinite(s) && s > 0.f; }
+
+// Causal schedule: heads per group so that about two waves of CTAs work on
+// the same few heads (their K/V stay in L2).
+int group_heads(int BH, int n_qpairs, int grid) {
+  int g = (2 * grid + n_qpairs - 1) / n_qpairs;
+  if (g < 1) g = 1;
+  if (g > BH) g = BH;
+  return g;
+}
+
+fa_status launch_attention(DeviceState* ds, int elem, const void* q, const void* k, const void* v, void* o,
+                           float* lse, const float* q_scale, const float* k_scale, int BH, int N, int d,
+                           float softmax_scale, int causal, cudaStream_t stream) {
+  fa::FwdLaunch l;
+  const int qk_bytes = elem == fa::kElemE4M3 ? 1 : 2;
+  fa_status st;
+  const bool fp16 = elem == fa::kElemF16;
+  if ((st = make_map(&l.map_q, q, BH, N, d, qk_bytes, fp16)) != FA_OK) return st;
+  if ((st = make_map(&l.map_k, k, BH, N, d, qk_bytes, fp16)) != FA_OK) return st;
+  if ((st = make_map(&l.map_v, v, BH, N, d, 2, fp16)) != FA_OK) return st;
+  fa::FwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.o = o;
+  a.lse = lse;
+  a.q_scale = q_scale;
+  a.k_scale = k_scale;
+  a.status = ds->status;
+  a.BH = BH;
+  a.N = N;
+  a.n_qpairs = (N + 255) / 256;
+  a.n_work = BH * a.n_qpairs;
+  a.n_qtiles = (N + 127) / 128;
+  a.causal = causal ? 1 : 0;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.wait_limit_ns = g_wait_ns;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    a.withhold = g_withhold;
+    g_withhold = 0;
+  }
+  l.grid = a.n_work < ds->sms ? a.n_work : ds->sms;
+  a.group_heads = group_heads(BH, a.n_qpairs, l.grid);
+  l.args = &a;
+  l.stream = stream;
+  cudaError_t e;
+  if (elem == fa::kElemBF16)
+    e = fa::launch_fwd_bf16(d, l);
+  else if (elem == fa::kElemF16)
+    e = fa::launch_fwd_f16(d, l);
+  else
+    e = fa::launch_fwd_e4m3(d, l);
+  return map_cuda(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                 float softmax_scale, int causal, fa_dtype dtype, void* stream) {
+  if (dtype != FA_BF16 && dtype != FA_FP16 && dtype != FA_E4M3) return FA_ERR_INVALID;
+  fa_status st = check_shape(B, H, N, d);
+  if (st != FA_OK) return st;
+  if (dtype == FA_E4M3 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o) return FA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)))
+    return FA_ERR_INVALID;
+  if (!scale_ok(softmax_scale) || (causal != 0 && causal != 1)) return FA_ERR_INVALID;
+  if (o == q || o == k || o == v) return FA_ERR_INVALID;
+
+  DeviceState* ds = nullptr;
+  if ((st = device_state(&ds)) != FA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  if (dtype == FA_BF16) return launch_attention(ds, fa::kElemBF16, q, k, v, o, lse, nullptr, nullptr, BH, N, d,
+                                                softmax_scale, causal, s);
+  if (dtype == FA_FP16) return launch_attention(ds, fa::kElemF16, q, k, v, o, lse, nullptr, nullptr, BH, N, d,
+                                                softmax_scale, causal, s);
+
+  // FA_E4M3: quantise q and k into the library workspace, then attend.
+  const size_t elems = static_cast<size_t>(BH) * N * d;
+  const size_t n_scales = static_cast<size_t>(BH) * ((N + 127) / 128);
+  const size_t codes_bytes = (elems + 255) & ~static_cast<size_t>(255);
+  const size_t need = 2 * codes_bytes + 2 * n_scales * sizeof(float);
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (ds->ws_bytes < need) {
+      if (ds->ws) cudaFree(ds->ws);
+      ds->ws = nullptr;
+      ds->ws_bytes = 0;
+      if (cudaMalloc(&ds->ws, need) != cudaSuccess) return FA_ERR_CUDA;
+      ds->ws_bytes = need;
+    }
+  }
+  uint8_t* q8 = static_cast<uint8_t*>(ds->ws);
+  uint8_t* k8 = q8 + codes_bytes;
+  float* qs = reinterpret_cast<float*>(k8 + codes_bytes);
+  float* ks = qs + n_scales;
+  if (fa::launch_quantize_e4m3(q, q8, qs, BH, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (fa::launch_quantize_e4m3(k, k8, ks, BH, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
+  return launch_attention(ds, fa::kElemE4M3, q8, k8, v, o, lse, qs, ks, BH, N, d, softmax_scale, causal, s);
+}
+
+fa_status fa_quantize_e4m3(const void* x, void* x8, float* scales, int B, int H, int N, int d, void* stream) {
+  fa_status st = check_shape(B, H, N, d);
+  if (st != FA_OK) return st;
+  if (!x || !x8 || !scales) return FA_ERR_INVALID;
+  if (!aligned16(x) || !aligned16(x8) || !aligned16(scales)) return FA_ERR_INVALID;
+  DeviceState* ds = nullptr;
+  if ((st = device_state(&ds)) != FA_OK) return st;
+  return map_cuda(fa::launch_quantize_e4m3(x, x8, scales, B * H, N, d, static_cast<cudaStream_t>(stream)));
+}
+
+fa_status fa_fwd_fp8(const void* q8, const float* q_scale, const void* k8, const float* k_scale, const void* v,
+                     void* o, float* lse, int B, int H, int N, int d, float softmax_scale, int causal,
+                     void* stream) {
+  fa_status st = check_shape(B, H, N, d);
+  if (st != FA_OK) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (!q8 || !k8 || !q_scale || !k_scale || !v || !o) return FA_ERR_INVALID;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)))
+    return FA_ERR_INVALID;
+  if ((reinterpret_cast<uintptr_t>(q_scale) & 3u) || (reinterpret_cast<uintptr_t>(k_scale) & 3u))
+    return FA_ERR_INVALID;
+  if (!scale_ok(softmax_scale) || (causal != 0 && causal != 1)) return FA_ERR_INVALID;
+  if (o == q8 || o == k8 || o == v) return FA_ERR_INVALID;
+  DeviceState* ds = nullptr;
+  if ((st = device_state(&ds)) != FA_OK) return st;
+  return launch_attention(ds, fa::kElemE4M3, q8, k8, v, o, lse, q_scale, k_scale, B * H, N, d, softmax_scale,
+                          causal, static_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_last_device_status(void* stream) {
+  DeviceState* ds = nullptr;
+  fa_status st = device_state(&ds);
+  if (st != FA_OK) return st;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpy(&word, ds->status, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return FA_ERR_CUDA;
+  if (word != 0 && cudaMemset(ds->status, 0, sizeof(word)) != cudaSuccess) return FA_ERR_CUDA;
+  return word ? FA_ERR_TIMEOUT : FA_OK;
+}
+
+const char* fa_status_string(fa_status status) {
+  switch (status) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported head dimension or dtype";
+    case FA_ERR_ARCH: return "device is not compute capability 10.x (sm_100)";
+    case FA_ERR_CUDA: return "CUDA call or kernel launch failed";
+    case FA_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
+    default: return "unknown status";
+  }
+}
+
+fa_status fa_release(void) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& s = g_dev[dev];
+  if (s.ws) cudaFree(s.ws);
+  if (s.status) cudaFree(s.status);
+  s = DeviceState();
+  return FA_OK;
+}
+
+fa_status fa_debug_set_wait_limit(uint64_t nanoseconds) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_wait_ns = nanoseconds ? nanoseconds : kDefaultWaitNs;
+  return FA_OK;
+}
+
+fa_status fa_debug_withhold_arrival(int enable) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_withhold = enable ? 1 : 0;
+  return FA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,33 @@
+// fa_fwd_16bit.cu — bf16 and fp16 instantiations of the forward kernel.
+#include "fa_fwd_launch.cuh"
+
+namespace fa {
+
+cudaError_t launch_fwd_bf16(int d, const FwdLaunch& l) {
+  switch (d) {
+    case 32: return launch_fwd_t<32, kElemBF16>(l);
+    case 64: return launch_fwd_t<64, kElemBF16>(l);
+    case 128: return launch_fwd_t<128, kElemBF16>(l);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_fwd_f16(int d, const FwdLaunch& l) {
+  switch (d) {
+    case 32: return launch_fwd_t<32, kElemF16>(l);
+    case 64: return launch_fwd_t<64, kElemF16>(l);
+    case 128: return launch_fwd_t<128, kElemF16>(l);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+int fwd_smem_bytes(int d, int elem) {
+  if (elem == kElemE4M3) return FwdCfg<128, kElemE4M3>::SMEM_BYTES;
+  switch (d) {
+    case 32: return FwdCfg<32, kElemBF16>::SMEM_BYTES;
+    case 64: return FwdCfg<64, kElemBF16>::SMEM_BYTES;
+    default: return FwdCfg<128, kElemBF16>::SMEM_BYTES;
+  }
+}
+
+}  // namespace fa

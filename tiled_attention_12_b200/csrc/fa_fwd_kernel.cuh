@@ -1,0 +1,553 @@
+// fa_fwd_kernel.cuh — persistent, warp-specialised attention forward for sm_100a.
+//
+// Computes O = softmax(scale * Q K^T [+ causal]) V and LSE = log sum exp per
+// row, tile by tile with the online-softmax recurrence, so the N x N scores
+// never leave the SM ("从理论到实现：基于Triton剖析FlashAttention三代的演进与优化"
+// §2.1 for the recurrence, §3.1 for the block causal mask, §4.1 for FP8 scores
+// with dynamic scales, §4.2 for loads prefetched while the previous tile
+// computes; the "Flash Attention" tag page, excerpt "注意力计算的性能瓶颈",
+// for the Q-outer / K,V-inner order of FlashAttention V2 and the single
+// division by l at the end).
+//
+// One CTA per SM (512 TMEM columns), looping over work tiles.  A work tile is
+// 256 consecutive query rows of one (batch, head): two 128-row Q tiles, each
+// owned by one softmax warpgroup, that share every K/V tile loaded.
+//
+//   warps 0-3  softmax warpgroup 0 (Q tile 0): scores -> P, running m and l,
+//              O rescale, epilogue (O / l, LSE)
+//   warps 4-7  softmax warpgroup 1 (Q tile 1)
+//   warp  8    MMA issuer (one thread): S_i = Q_i K^T and O_i += P_i V on the
+//              tensor cores, accumulators in tensor memory
+//   warp  9    TMA producer (one thread): Q tiles and a ring of K/V tiles
+//
+// Tensor memory (512 fp32 columns x 128 lanes, lane = query row):
+//   S_0 [0,128)  S_1 [128,256)  O_0 [256,256+D)  O_1 [256+D,256+2D)
+//   P_i (16-bit) overwrites the first 64 columns of S_i once S_i is read.
+//
+// MMA order per K/V step j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1).  While one
+// warpgroup exponentiates its scores, the tensor cores run the other Q tile's
+// products.  tcgen05.mma operations issued by one thread execute in issue
+// order, so S_i(j+1) may overwrite P_i(j) after PV_i(j) is issued, and the
+// completion of S_i(j+1) also tells its warpgroup that PV_i(j) is finished
+// (the O rescale for step j+1 needs that).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <type_traits>
+
+#include "ptx.cuh"
+
+namespace fa {
+
+enum : int { kElemBF16 = 0, kElemF16 = 1, kElemE4M3 = 2 };
+
+// Status bits written to the device status word when a wait gives up.
+enum : unsigned { kStatusProducer = 1u, kStatusMma = 2u, kStatusSoftmax = 4u, kStatusDrain = 8u };
+
+struct FwdArgs {
+  void* o;                 // [BH, N, D], element type of V
+  float* lse;              // [BH, N] fp32 or nullptr
+  const float* q_scale;    // [BH, ceil(N/128)] (e4m3 only)
+  const float* k_scale;    // [BH, ceil(N/128)] (e4m3 only)
+  unsigned int* status;    // device status word
+  int BH;                  // batch * heads
+  int N;                   // sequence length
+  int n_qpairs;            // ceil(N / 256): work tiles per head
+  int n_work;              // BH * n_qpairs
+  int causal;
+  int group_heads;         // causal schedule: heads per group
+  int withhold;            // test hook: skip the first K/V load
+  int n_qtiles;            // ceil(N / 128): scale entries per head
+  float scale_log2;        // softmax_scale * log2(e)
+  uint64_t wait_limit_ns;  // bound for every in-kernel wait
+};
+
+template <int D, int ELEM>
+struct FwdCfg {
+  static constexpr int BM = 128;  // query rows per Q tile = MMA M
+  static constexpr int BN = 128;  // keys per K/V tile = S MMA N
+  static constexpr int QK_BYTES = (ELEM == kElemE4M3) ? 1 : 2;
+  static constexpr int QK_ROW = D * QK_BYTES;
+  static constexpr int V_ROW = D * 2;
+  static constexpr int SW_QK = QK_ROW >= 128 ? 128 : QK_ROW;  // swizzle span in bytes
+  static constexpr int SW_V = V_ROW >= 128 ? 128 : V_ROW;
+  static_assert(SW_QK == 128 || SW_QK == 64, "head dim gives an unsupported swizzle span");
+  static_assert(SW_V == 128 || SW_V == 64, "head dim gives an unsupported swizzle span");
+  static constexpr int Q_TILE = BM * QK_ROW;
+  static constexpr int K_TILE = BN * QK_ROW;
+  static constexpr int V_TILE = BN * V_ROW;
+  static constexpr int STAGE = K_TILE > V_TILE ? K_TILE : V_TILE;
+  static constexpr int NS_FIT = (200 * 1024 - 2 * Q_TILE) / STAGE;
+  static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;  // K/V ring depth
+  static_assert(NS >= 2, "ring too shallow");
+  static constexpr int TILE_BYTES = 2 * Q_TILE + NS * STAGE;
+  static constexpr int NUM_BARS = 2 + 2 + 2 * NS + 2 + 2 + 2 + 1;
+  // at least 120 KB so that two CTAs never share an SM (each holds all 512
+  // tensor-memory columns; a second resident CTA would only wait)
+  static constexpr int SMEM_NEED = 1024 + TILE_BYTES + 8 * NUM_BARS;
+  static constexpr int SMEM_BYTES = SMEM_NEED > 120 * 1024 ? SMEM_NEED : 120 * 1024;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget exceeded");
+  static constexpr int K_STEPS_QK = QK_ROW / 32;   // 32 bytes of K per S MMA (16 x 16-bit or 32 x 8-bit)
+  static constexpr int K_STEPS_PV = BN / 16;       // 16 keys per P V MMA
+  static constexpr int THREADS = 320;
+  static constexpr int MMA_WARP = 8;
+  static constexpr int LOAD_WARP = 9;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t S_COL0 = 0, S_COL1 = 128, O_COL0 = 256, O_COL1 = 256 + D;
+  static_assert(O_COL1 + D <= TMEM_COLS, "tensor memory budget exceeded");
+  static constexpr uint32_t IDESC_QK =
+      instr_desc(ELEM == kElemBF16 ? 1u : 0u, ELEM == kElemBF16 ? 1u : 0u, 0u, BM, BN);
+  static constexpr uint32_t IDESC_PV =
+      instr_desc(ELEM == kElemF16 ? 0u : 1u, ELEM == kElemF16 ? 0u : 1u, 1u, BM, D);
+  static constexpr uint32_t SWZ_QK = SW_QK == 128 ? 2u : 4u;
+  static constexpr uint32_t SWZ_V = SW_V == 128 ? 2u : 4u;
+  static constexpr float TAU = 8.0f;  // deferred-rescale threshold (log2 units)
+};
+
+struct Barriers {
+  uint64_t* q_full;    // [2]  TMA -> MMA
+  uint64_t* q_empty;   // [2]  MMA -> TMA
+  uint64_t* kv_full;   // [NS] TMA -> MMA
+  uint64_t* kv_empty;  // [NS] MMA -> TMA
+  uint64_t* s_full;    // [2]  MMA -> softmax i
+  uint64_t* p_full;    // [2]  softmax i -> MMA (4 warp arrivals)
+  uint64_t* o_full;    // [2]  MMA -> softmax i (epilogue)
+  uint64_t* mma_done;  // [1]  MMA drain
+};
+
+struct WorkTile {
+  int bh;
+  int tp;  // index of the 256-row query block within the head
+};
+
+// Work order.  Non-causal: head-major (consecutive CTAs share a head's K/V in
+// L2).  Causal: heads in groups of `group_heads`; inside a group the longest
+// tiles (largest tp) come first, so the static round-robin hand-out finishes
+// with the short ones.
+__device__ __forceinline__ WorkTile decode_work(const FwdArgs& a, int w) {
+  WorkTile t;
+  if (!a.causal) {
+    t.bh = w / a.n_qpairs;
+    t.tp = w - t.bh * a.n_qpairs;
+  } else {
+    const int per_group = a.group_heads * a.n_qpairs;
+    const int g = w / per_group;
+    const int rem = w - g * per_group;
+    const int left = a.BH - g * a.group_heads;
+    const int heads = left < a.group_heads ? left : a.group_heads;
+    const int level = rem / heads;
+    t.bh = g * a.group_heads + (rem - level * heads);
+    t.tp = a.n_qpairs - 1 - level;
+  }
+  return t;
+}
+
+// Number of K/V tiles a 128-row Q tile starting at q_start visits (0 when the
+// tile is entirely past the end of the sequence).  Causal: through the tile
+// holding the diagonal; tiles wholly above the diagonal are never issued.
+__device__ __forceinline__ int kv_tiles(const FwdArgs& a, int q_start) {
+  if (q_start >= a.N) return 0;
+  const int all = (a.N + 127) >> 7;
+  if (!a.causal) return all;
+  const int c = (q_start >> 7) + 1;
+  return c < all ? c : all;
+}
+
+__device__ __forceinline__ void record_failure(const FwdArgs& a, volatile int* abort_flag, unsigned bit) {
+  *abort_flag = 1;
+  atomicOr(a.status, bit);
+}
+
+template <int D, int ELEM>
+__global__ void __launch_bounds__(320, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                  const __grid_constant__ CUtensorMap map_v, const FwdArgs a) {
+  using C = FwdCfg<D, ELEM>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint32_t tmem_holder;
+  __shared__ int abort_flag_storage;
+  volatile int* abort_flag = &abort_flag_storage;
+
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* sQ = base;                       // [2][Q_TILE]
+  uint8_t* sKV = base + 2 * C::Q_TILE;      // [NS][STAGE]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + C::TILE_BYTES);
+  Barriers b;
+  b.q_full = bars;
+  b.q_empty = bars + 2;
+  b.kv_full = bars + 4;
+  b.kv_empty = bars + 4 + C::NS;
+  b.s_full = bars + 4 + 2 * C::NS;
+  b.p_full = b.s_full + 2;
+  b.o_full = b.p_full + 2;
+  b.mma_done = b.o_full + 2;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    abort_flag_storage = 0;
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&b.q_full[i], 1);
+      mbar_init(&b.q_empty[i], 1);
+      mbar_init(&b.s_full[i], 1);
+      mbar_init(&b.p_full[i], 4);
+      mbar_init(&b.o_full[i], 1);
+    }
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(&b.kv_full[s], 1);
+      mbar_init(&b.kv_empty[s], 1);
+    }
+    mbar_init(b.mma_done, 1);
+    fence_barrier_init();
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(&tmem_holder, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_holder;
+  const uint64_t limit = a.wait_limit_ns;
+
+  if (warp == C::LOAD_WARP) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&map_q);
+      tma_prefetch_desc(&map_k);
+      tma_prefetch_desc(&map_v);
+      int kv_it = 0;
+      int q_use[2] = {0, 0};
+      int last_round[C::NS];
+#pragma unroll
+      for (int s = 0; s < C::NS; ++s) last_round[s] = -1;
+      bool withhold = a.withhold != 0;
+      auto run = [&]() -> bool {
+        for (int w = blockIdx.x; w < a.n_work; w += gridDim.x) {
+          const WorkTile t = decode_work(a, w);
+          const int q0 = t.tp * 256;
+          const int n[2] = {kv_tiles(a, q0), kv_tiles(a, q0 + 128)};
+          for (int i = 0; i < 2; ++i) {
+            if (n[i] == 0) continue;
+            if (q_use[i] > 0 && !wait_bounded(&b.q_empty[i], (q_use[i] - 1) & 1, abort_flag, limit))
+              return false;
+            mbar_arrive_expect_tx(&b.q_full[i], C::Q_TILE);
+#pragma unroll
+            for (int c = 0; c < C::QK_ROW / C::SW_QK; ++c)
+              tma_load_3d(sQ + i * C::Q_TILE + c * C::BM * C::SW_QK, &map_q, &b.q_full[i],
+                          c * (C::SW_QK / C::QK_BYTES), q0 + i * 128, t.bh);
+            ++q_use[i];
+          }
+          const int nkv = n[0] > n[1] ? n[0] : n[1];
+          for (int j = 0; j < nkv; ++j) {
+#pragma unroll
+            for (int kind = 0; kind < 2; ++kind) {
+              const int s = kv_it % C::NS;
+              const int r = kv_it / C::NS;
+              if (r > 0 && !wait_bounded(&b.kv_empty[s], (r - 1) & 1, abort_flag, limit)) return false;
+              ++kv_it;
+              if (withhold) {  // test hook: this tile never arrives
+                withhold = false;
+                continue;
+              }
+              uint8_t* dst = sKV + s * C::STAGE;
+              if (kind == 0) {
+                mbar_arrive_expect_tx(&b.kv_full[s], C::K_TILE);
+#pragma unroll
+                for (int c = 0; c < C::QK_ROW / C::SW_QK; ++c)
+                  tma_load_3d(dst + c * C::BN * C::SW_QK, &map_k, &b.kv_full[s], c * (C::SW_QK / C::QK_BYTES),
+                              j * 128, t.bh);
+              } else {
+                mbar_arrive_expect_tx(&b.kv_full[s], C::V_TILE);
+#pragma unroll
+                for (int c = 0; c < C::V_ROW / C::SW_V; ++c)
+                  tma_load_3d(dst + c * C::BN * C::SW_V, &map_v, &b.kv_full[s], c * (C::SW_V / 2), j * 128, t.bh);
+              }
+              last_round[s] = r;
+            }
+          }
+        }
+        return true;
+      };
+      if (!run()) record_failure(a, abort_flag, kStatusProducer);
+      // Drain: every bulk copy this thread issued has landed before the CTA
+      // may exit (normal completion finds these phases already complete).
+      volatile int never = 0;
+      bool drained = true;
+      for (int i = 0; i < 2; ++i)
+        if (q_use[i] > 0) drained &= wait_bounded(&b.q_full[i], (q_use[i] - 1) & 1, &never, limit);
+#pragma unroll
+      for (int s = 0; s < C::NS; ++s)
+        if (last_round[s] >= 0) drained &= wait_bounded(&b.kv_full[s], last_round[s] & 1, &never, limit);
+      if (!drained) atomicOr(a.status, kStatusDrain);
+    }
+  } else if (warp == C::MMA_WARP) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t sQ_addr = smem_u32(sQ);
+      const uint32_t sKV_addr = smem_u32(sKV);
+      int kv_it = 0;
+      int q_use[2] = {0, 0};
+      int p_cnt[2] = {0, 0};
+
+      auto issue_s = [&](int i, int stage) {
+        const uint32_t d_tmem = tmem + (i ? C::S_COL1 : C::S_COL0);
+        const uint32_t qa = sQ_addr + i * C::Q_TILE;
+        const uint32_t ka = sKV_addr + stage * C::STAGE;
+#pragma unroll
+        for (int kk = 0; kk < C::K_STEPS_QK; ++kk) {
+          const uint32_t byte = kk * 32;
+          const uint32_t off = (byte / C::SW_QK) * (C::BM * C::SW_QK) + (byte % C::SW_QK);
+          const uint64_t ad = smem_desc(qa + off, 16, 8 * C::SW_QK, C::SWZ_QK);
+          const uint64_t bd = smem_desc(ka + off, 16, 8 * C::SW_QK, C::SWZ_QK);
+          if constexpr (ELEM == kElemE4M3)
+            mma_f8_ss(d_tmem, ad, bd, C::IDESC_QK, kk > 0);
+          else
+            mma_f16_ss(d_tmem, ad, bd, C::IDESC_QK, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int i, int stage, bool accumulate) {
+        const uint32_t d_tmem = tmem + (i ? C::O_COL1 : C::O_COL0);
+        const uint32_t p_tmem = tmem + (i ? C::S_COL1 : C::S_COL0);
+        const uint32_t va = sKV_addr + stage * C::STAGE;
+#pragma unroll
+        for (int kk = 0; kk < C::K_STEPS_PV; ++kk) {
+          const uint64_t bd = smem_desc(va + kk * 16 * C::SW_V, C::BN * C::SW_V, 8 * C::SW_V, C::SWZ_V);
+          mma_f16_ts(d_tmem, p_tmem + kk * 8, bd, C::IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
+        }
+      };
+      auto acquire = [&](int& stage) -> bool {
+        stage = kv_it % C::NS;
+        const int r = kv_it / C::NS;
+        ++kv_it;
+        if (!wait_bounded(&b.kv_full[stage], r & 1, abort_flag, limit)) return false;
+        tc_fence_after();
+        return true;
+      };
+
+      auto run = [&]() -> bool {
+        for (int w = blockIdx.x; w < a.n_work; w += gridDim.x) {
+          const WorkTile t = decode_work(a, w);
+          const int q0 = t.tp * 256;
+          const int n0 = kv_tiles(a, q0), n1 = kv_tiles(a, q0 + 128);
+          const int nkv = n0 > n1 ? n0 : n1;
+          if (n0 > 0) {
+            if (!wait_bounded(&b.q_full[0], q_use[0] & 1, abort_flag, limit)) return false;
+            ++q_use[0];
+          }
+          if (n1 > 0) {
+            if (!wait_bounded(&b.q_full[1], q_use[1] & 1, abort_flag, limit)) return false;
+            ++q_use[1];
+          }
+          int sk;
+          if (!acquire(sk)) return false;
+          if (n0 > 0) {
+            issue_s(0, sk);
+            tc_commit(&b.s_full[0]);
+            if (n0 == 1) tc_commit(&b.q_empty[0]);
+          }
+          if (n1 > 0) {
+            issue_s(1, sk);
+            tc_commit(&b.s_full[1]);
+            if (n1 == 1) tc_commit(&b.q_empty[1]);
+          }
+          tc_commit(&b.kv_empty[sk]);
+          for (int j = 0; j < nkv; ++j) {
+            int sv;
+            if (!acquire(sv)) return false;
+            if (j < n0) {
+              if (!wait_bounded(&b.p_full[0], p_cnt[0] & 1, abort_flag, limit)) return false;
+              ++p_cnt[0];
+              tc_fence_after();
+              issue_pv(0, sv, j > 0);
+              if (j == n0 - 1) tc_commit(&b.o_full[0]);
+            }
+            const bool next = j + 1 < nkv;
+            int sk2 = 0;
+            if (next) {
+              if (!acquire(sk2)) return false;
+              if (j + 1 < n0) {
+                issue_s(0, sk2);
+                tc_commit(&b.s_full[0]);
+                if (j + 1 == n0 - 1) tc_commit(&b.q_empty[0]);
+              }
+            }
+            if (j < n1) {
+              if (!wait_bounded(&b.p_full[1], p_cnt[1] & 1, abort_flag, limit)) return false;
+              ++p_cnt[1];
+              tc_fence_after();
+              issue_pv(1, sv, j > 0);
+              if (j == n1 - 1) tc_commit(&b.o_full[1]);
+            }
+            tc_commit(&b.kv_empty[sv]);
+            if (next) {
+              if (j + 1 < n1) {
+                issue_s(1, sk2);
+                tc_commit(&b.s_full[1]);
+                if (j + 1 == n1 - 1) tc_commit(&b.q_empty[1]);
+              }
+              tc_commit(&b.kv_empty[sk2]);
+            }
+          }
+        }
+        return true;
+      };
+      if (!run()) record_failure(a, abort_flag, kStatusMma);
+      // Drain: all issued MMAs complete before tensor memory is released.
+      tc_commit(b.mma_done);
+      volatile int never = 0;
+      if (!wait_bounded(b.mma_done, 0, &never, limit)) atomicOr(a.status, kStatusDrain);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int wg = warp >> 2;            // which Q tile
+    const int wq = warp & 3;             // warp within the warpgroup -> TMEM lanes
+    const int row = wq * 32 + lane;      // query row within the Q tile
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t t_s = tmem + lane_off + (wg ? C::S_COL1 : C::S_COL0);
+    const uint32_t t_o = tmem + lane_off + (wg ? C::O_COL1 : C::O_COL0);
+    uint64_t* s_full = &b.s_full[wg];
+    uint64_t* p_full = &b.p_full[wg];
+    uint64_t* o_full = &b.o_full[wg];
+    int s_cnt = 0, o_cnt = 0;
+    using OutT = typename std::conditional<ELEM == kElemF16, __half, __nv_bfloat16>::type;
+
+    auto wait_warp = [&](uint64_t* bar, int parity) -> bool {
+      bool ok = wait_bounded(bar, parity & 1, abort_flag, limit);
+      return __all_sync(0xffffffffu, ok);
+    };
+
+    auto run = [&]() -> bool {
+      for (int w = blockIdx.x; w < a.n_work; w += gridDim.x) {
+        const WorkTile t = decode_work(a, w);
+        const int q_start = t.tp * 256 + wg * 128;
+        const int nkv = kv_tiles(a, q_start);
+        if (nkv == 0) continue;
+        const int qrow = q_start + row;
+        float sl2_q = a.scale_log2;
+        if constexpr (ELEM == kElemE4M3) sl2_q = a.scale_log2 / a.q_scale[t.bh * a.n_qtiles + (q_start >> 7)];
+        float m = -INFINITY;  // running max, log2 units of the scaled score
+        float l = 0.f;        // running sum of exponentials
+        for (int j = 0; j < nkv; ++j) {
+          if (!wait_warp(s_full, s_cnt)) return false;
+          ++s_cnt;
+          tc_fence_after();
+          float sl2 = sl2_q;
+          if constexpr (ELEM == kElemE4M3) sl2 = sl2_q / a.k_scale[t.bh * a.n_qtiles + j];
+          uint32_t sr[4][32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, sr[c]);
+          tmem_ld_wait(sr[0]);
+          reg_tie(sr[1]);
+          reg_tie(sr[2]);
+          reg_tie(sr[3]);
+#define FA_S(c) __uint_as_float(sr[(c) >> 5][(c) & 31])
+          if (j == nkv - 1) {
+            // last tile of this row block: keys past the sequence end, and
+            // (causal) keys after the query, become -inf
+            int limit_key = a.N - 1;
+            if (a.causal && qrow < limit_key) limit_key = qrow;
+            const int kbase = j * 128;
+#pragma unroll
+            for (int c = 0; c < 128; ++c)
+              if (kbase + c > limit_key) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+          }
+          float mx0 = FA_S(0), mx1 = FA_S(1), mx2 = FA_S(2), mx3 = FA_S(3);
+#pragma unroll
+          for (int c = 4; c < 128; c += 4) {
+            mx0 = fmaxf(mx0, FA_S(c));
+            mx1 = fmaxf(mx1, FA_S(c + 1));
+            mx2 = fmaxf(mx2, FA_S(c + 2));
+            mx3 = fmaxf(mx3, FA_S(c + 3));
+          }
+          const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+          if (j == 0) {
+            m = mx;
+          } else {
+            const bool need = mx - m > C::TAU;
+            if (__any_sync(0xffffffffu, need)) {
+              const float m_new = fmaxf(m, mx);
+              const float alpha = ex2_approx(m - m_new);
+              m = m_new;
+              l *= alpha;
+#pragma unroll
+              for (int c = 0; c < D / 32; ++c) {
+                uint32_t orr[32];
+                tmem_ld32(t_o + c * 32, orr);
+                tmem_ld_wait(orr);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+                tmem_st32(t_o + c * 32, orr);
+              }
+            }
+          }
+          const float neg_m = -m;
+          float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float p0 = ex2_approx(fmaf(FA_S(c * 32 + 2 * e), sl2, neg_m));
+              const float p1 = ex2_approx(fmaf(FA_S(c * 32 + 2 * e + 1), sl2, neg_m));
+              sum0 += p0;
+              sum1 += p1;
+              if constexpr (ELEM == kElemF16)
+                pk[e] = pack_f16x2(p0, p1);
+              else
+                pk[e] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(t_s + c * 16, pk);
+          }
+#undef FA_S
+          l += sum0 + sum1;
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(p_full);
+        }
+        // epilogue: O / l -> global, LSE
+        if (!wait_warp(o_full, o_cnt)) return false;
+        ++o_cnt;
+        tc_fence_after();
+        const float inv_l = 1.f / l;
+        OutT* orow = reinterpret_cast<OutT*>(a.o) + (static_cast<size_t>(t.bh) * a.N + qrow) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t orr[32];
+          tmem_ld32(t_o + c * 32, orr);
+          tmem_ld_wait(orr);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float v0 = __uint_as_float(orr[2 * e]) * inv_l;
+            const float v1 = __uint_as_float(orr[2 * e + 1]) * inv_l;
+            pk[e] = (ELEM == kElemF16) ? pack_f16x2(v0, v1) : pack_bf16x2(v0, v1);
+          }
+          if (qrow < a.N) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
+        }
+        if (a.lse != nullptr && qrow < a.N)
+          a.lse[static_cast<size_t>(t.bh) * a.N + qrow] = (m + __log2f(l)) * 0.69314718055994531f;
+      }
+      return true;
+    };
+    if (!run()) record_failure(a, abort_flag, kStatusSoftmax);
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,20 @@
+// fa_fwd_launch.cuh — launches one instantiation of the forward kernel.
+#pragma once
+
+#include "fa_fwd_kernel.cuh"
+#include "fa_launch.h"
+
+namespace fa {
+
+template <int D, int ELEM>
+cudaError_t launch_fwd_t(const FwdLaunch& l) {
+  using C = FwdCfg<D, ELEM>;
+  auto kernel = fa_fwd_kernel<D, ELEM>;
+  // The attribute is per device; setting it again is harmless.
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  kernel<<<l.grid, C::THREADS, C::SMEM_BYTES, l.stream>>>(l.map_q, l.map_k, l.map_v, *l.args);
+  return cudaGetLastError();
+}
+
+}  // namespace fa

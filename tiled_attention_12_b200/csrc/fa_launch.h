@@ -1,0 +1,29 @@
+// fa_launch.h — host-side launch interface between the C ABI (fa_api.cu) and
+// the translation units that hold the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace fa {
+
+struct FwdArgs;
+
+struct FwdLaunch {
+  CUtensorMap map_q, map_k, map_v;
+  const FwdArgs* args;
+  int grid;
+  cudaStream_t stream;
+};
+
+// Returns cudaSuccess once the kernel is enqueued.
+cudaError_t launch_fwd_bf16(int d, const FwdLaunch& l);
+cudaError_t launch_fwd_f16(int d, const FwdLaunch& l);
+cudaError_t launch_fwd_e4m3(int d, const FwdLaunch& l);
+cudaError_t launch_quantize_e4m3(const void* x, void* x8, float* scales, int BH, int N, int d,
+                                 cudaStream_t stream);
+int fwd_smem_bytes(int d, int elem);
+
+}  // namespace fa
