@@ -1,0 +1,465 @@
+"""Benchmark: attention forward TFLOPS on B200, one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference] [--no-suite] [--no-e2e]
+
+A step is one pass of the forward over every case of the workload (default
+"dmodel512_h16": d_model = 512 with 16 heads, B=1, H=16, d=32, N in {1024,
+16384}, causal and non-causal).  Inputs are resident in HBM when the timed
+region starts; the L2 cache is flushed (a 512 MiB write) before every step and
+each step is timed on its own with CUDA events on the launching stream.
+
+With N GPUs (torchrun, one process per GPU) every rank runs the same
+per-GPU workload on its own batch (independent problems, no collective on the
+data path): weak scaling, value = all ranks' FLOPs / max over ranks of time.
+
+--impl reference times the fp64 CPU oracle (the only other implementation of
+this method here) on a bounded row sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd TFLOPS and % of B200 dense tensor peak (bf16; causal & non)"
+L2_FLUSH_BYTES = 512 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+EXP_PER_CLK_SM = 16          # ex2 results per clock per SM (special-function unit)
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--workload", default="dmodel512_h16")
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-suite", action="store_true", help="skip the per-workload suite")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu", action="store_true", help="skip the oracle baseline")
+    p.add_argument("--only-case", default=None, help="time one case of the workload (profiling)")
+    return p.parse_args()
+
+
+KERNEL_SOURCES = ("tiled_attention_12_b200/csrc/fa_fwd_kernel.cuh", "tiled_attention_12_b200/csrc/ptx.cuh",
+                  "tiled_attention_12_b200/csrc/fa_fwd_launch.cuh", "tiled_attention_12_b200/csrc/fa_api.cu")
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(case_name: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel sources changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "fa_fwd_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    entry = d.get("cases", {}).get(case_name)
+    return None if entry is None else entry.get("dram_bytes_per_launch")
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int, path: str | None):
+        self.proc = None
+        self.path = path or os.path.join("/tmp", f"fa_clocks_{os.getpid()}.csv")
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(device_index)], stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i].lower().startswith("active")})
+        sm = [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    import tiled_attention_12_b200 as fa
+    from tiled_attention_12_b200.synth import WORKLOADS
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    fa.load()
+    wl = WORKLOADS[args.workload]
+    if any(c.fp8 for c in wl.cases):
+        raise SystemExit("the bench workload must be a 16-bit one")
+    stream = torch.cuda.current_stream()
+
+    # inputs resident in HBM (same recipe as synth.make_qkv, drawn on the
+    # device with a rank-specific seed: each rank holds its own batch)
+    def device_inputs(case, salt=0):
+        g = torch.Generator(device=dev)
+        g.manual_seed(case.seed * 1009 + rank * 7919 + salt)
+        shape = (case.B, case.H, case.N, case.d)
+        return [(torch.randn(shape, generator=g, device=dev) * case.value_scale).to(torch.bfloat16)
+                for _ in range(3)]
+
+    cases = [c for c in wl.cases if args.only_case in (None, c.name)]
+    if not cases:
+        raise SystemExit(f"no case {args.only_case} in {wl.name}")
+    tensors = []
+    for c in cases:
+        q, k, v = device_inputs(c)
+        o = torch.empty_like(v)
+        lse = torch.empty((c.B, c.H, c.N), device=dev, dtype=torch.float32)
+        tensors.append((q, k, v, o, lse))
+    flush = torch.empty(L2_FLUSH_BYTES // 4, device=dev, dtype=torch.float32)
+
+    def step():
+        for c, (q, k, v, o, lse) in zip(cases, tensors):
+            fa.fa_fwd(q, k, v, o=o, lse=lse, causal=c.causal, softmax_scale=c.softmax_scale)
+
+    def launch_one(i):
+        c = cases[i]
+        q, k, v, o, lse = tensors[i]
+        fa.fa_fwd(q, k, v, o=o, lse=lse, causal=c.causal, softmax_scale=c.softmax_scale)
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if fa.fa_last_device_status() != 0:
+        raise SystemExit("device status reports a timed-out wait during warm-up")
+
+    # ---- timed region: K steps, L2 flushed before each, events per case
+    n_cases = len(cases)
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n_cases)] for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
+                           if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else None)
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    for s in range(args.steps):
+        flush.zero_()
+        for i in range(n_cases):
+            ev[s][i][0].record(stream)
+            launch_one(i)
+            ev[s][i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    status = fa.fa_last_device_status()
+    if status != 0:
+        raise SystemExit(f"device status {status} after the timed region")
+    per_case_ms = [[ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(args.steps)] for i in range(n_cases)]
+    total_ms = sum(sum(x) for x in per_case_ms)
+    t_max = total_ms
+    if dist is not None:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_max = float(t.item())
+    flops_step = sum(c.flops for c in cases)
+    value = world * flops_step * args.steps / (t_max * 1e-3) / 1e12
+
+    result = {"flops_step": flops_step, "t_ms": t_max, "value": value, "clocks": clocks,
+              "per_case_ms": per_case_ms}
+
+    # ---- dominant kernel (largest share of the step) for the roofline
+    mean_case = [sum(x) / len(x) for x in per_case_ms]
+    dom = max(range(n_cases), key=lambda i: mean_case[i])
+    result["dominant"] = (cases[dom], mean_case[dom])
+    result["cases"] = {c.name: {"ms": round(mean_case[i], 5), "tflops": round(c.flops / mean_case[i] / 1e9, 2)}
+                       for i, c in enumerate(cases)}
+
+    # ---- end to end through the public API with host buffers
+    if not args.no_e2e:
+        host = []
+        for c, (q, k, v, o, lse) in zip(cases, tensors):
+            hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+            ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+            hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+            host.append((hq, hk, hv, ho, hl))
+        h2d = sum(t.numel() * t.element_size() for hq, hk, hv, _, _ in host for t in (hq, hk, hv))
+        d2h = sum(t.numel() * t.element_size() for _, _, _, ho, hl in host for t in (ho, hl))
+
+        def e2e_step():
+            for c, (q, k, v, o, lse), (hq, hk, hv, ho, hl) in zip(cases, tensors, host):
+                q.copy_(hq, non_blocking=True)
+                k.copy_(hk, non_blocking=True)
+                v.copy_(hv, non_blocking=True)
+                fa.fa_fwd(q, k, v, o=o, lse=lse, causal=c.causal, softmax_scale=c.softmax_scale)
+                ho.copy_(o, non_blocking=True)
+                hl.copy_(lse, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        k_e2e = max(3, min(args.steps, 30))
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(k_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = e0.elapsed_time(e1)
+        if dist is not None:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        result["e2e"] = {"value": round(world * flops_step * k_e2e / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOPS",
+                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k_e2e}
+
+    # ---- per-workload suite (rank 0 only, single GPU numbers)
+    if not args.no_suite and rank == 0:
+        suite = {}
+        for name, w in WORKLOADS.items():
+            if name in (args.workload, "tiny"):
+                continue
+            for c in w.cases:
+                try:
+                    q, k, v = device_inputs(c, salt=1)
+                    o = torch.empty_like(v)
+                    lse = torch.empty((c.B, c.H, c.N), device=dev, dtype=torch.float32)
+                    kw = dict(o=o, lse=lse, causal=c.causal, softmax_scale=c.softmax_scale,
+                              dtype=fa.FA_E4M3 if c.fp8 else None)
+                    for _ in range(3):
+                        fa.fa_fwd(q, k, v, **kw)
+                    times = []
+                    for _ in range(5):
+                        flush.zero_()
+                        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                        a0.record(stream)
+                        fa.fa_fwd(q, k, v, **kw)
+                        a1.record(stream)
+                        torch.cuda.synchronize()
+                        times.append(a0.elapsed_time(a1))
+                    ms = statistics.median(times)
+                    suite[c.name] = {"ms": round(ms, 4), "tflops": round(c.flops / ms / 1e9, 1),
+                                     "note": "includes e4m3 quantiser" if c.fp8 else ""}
+                    del q, k, v, o, lse
+                except Exception as e:  # report, never hide
+                    suite[c.name] = {"error": str(e)[:200]}
+        torch.cuda.synchronize()
+        if fa.fa_last_device_status() != 0:
+            raise SystemExit("device status reports a timed-out wait in the suite")
+        result["suite"] = suite
+    return result
+
+
+# ---------------------------------------------------------------- oracle
+def oracle_sample(cases, rows_per_case: int, head_of, workers=None):
+    """Times the fp64 oracle on a row sample; returns (flops, seconds)."""
+    import numpy as np
+
+    from oracle import attention_rows
+    from tiled_attention_12_b200.synth import make_qkv
+    import dataclasses
+
+    flops, secs = 0.0, 0.0
+    for c in cases:
+        h = head_of(c)
+        c1 = dataclasses.replace(c, H=1, seed=c.seed + 101 * h)
+        q, k, v = make_qkv(c1)
+        rows = np.unique(np.linspace(0, c.N - 1, min(c.N, rows_per_case)).astype(np.int64))
+        keys = (rows + 1) if c.causal else np.full(rows.shape, c.N)
+        flops += float(4.0 * c.d * keys.sum())
+        t0 = time.perf_counter()
+        attention_rows(q, k, v, c.softmax_scale, c.causal, 0, 0, rows)
+        secs += time.perf_counter() - t0
+    return flops, secs
+
+
+def cpu_baseline(cases):
+    """The oracle as it stands, on 3 heads' worth of full rows of every case."""
+    import dataclasses
+
+    from oracle import attention_ref
+    from tiled_attention_12_b200.synth import make_qkv
+
+    cores = os.cpu_count() or 1
+    flops, secs, heads = 0.0, 0.0, 5
+    for c in cases:
+        c1 = dataclasses.replace(c, H=heads)
+        q, k, v = make_qkv(c1)
+        t0 = time.perf_counter()
+        attention_ref(q, k, v, c.softmax_scale, c.causal, workers=cores)
+        secs += time.perf_counter() - t0
+        flops += c1.flops
+    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+            "sample": f"{heads} of {cases[0].H} heads of every case, all rows (fp64 numpy, {secs:.1f} s)"}
+
+
+def run_reference(args, rank, world):
+    from tiled_attention_12_b200.synth import WORKLOADS
+
+    wl = WORKLOADS[args.workload]
+    cases = list(wl.cases)
+    cores = os.cpu_count() or 1
+    rows = max(32, min(256, int(256 * 210 / max(1, args.steps + args.warmup))))
+    for i in range(args.warmup):
+        oracle_sample(cases, rows, lambda c, i=i: i % c.H)
+    flops, secs = 0.0, 0.0
+    for s in range(args.steps):
+        f, t = oracle_sample(cases, rows, lambda c, s=s: s % c.H)
+        flops += f
+        secs += t
+    value = flops / secs / 1e12
+    sample = f"{rows} evenly spaced query rows of one head per case per step (fp64 numpy oracle)"
+    line = {"metric": METRIC, "value": round(value, 6), "unit": "TFLOPS", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": wl.name, "description": wl.description,
+                       "cases": [c.name for c in cases], "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+    finally:
+        pass
+    if rank == 0:
+        from tiled_attention_12_b200.synth import WORKLOADS
+
+        peaks, peak_kind = load_peaks()
+        wl = WORKLOADS[args.workload]
+        run_cases = [c for c in wl.cases if args.only_case in (None, c.name)]
+        dom_case, dom_ms = res["dominant"]
+        achieved = dom_case.flops / (dom_ms * 1e-3) / 1e12
+        tensor_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        sm_mhz = float(peaks.get("sm_max_mhz", 1965.0))
+        n_sm = 148
+        # special-function-unit ceiling: one exp per score element, 4*d FLOPs per element
+        exp_peak = EXP_PER_CLK_SM * n_sm * sm_mhz * 1e6 * 4 * dom_case.d / 1e12
+        bound_alu = exp_peak < tensor_peak
+        roof = {"kernel": f"fa_fwd_kernel<{dom_case.d},bf16> ({dom_case.name})",
+                "bound": "alu" if bound_alu else "tensor",
+                "achieved": round(achieved, 2),
+                "peak": round(exp_peak if bound_alu else tensor_peak, 1),
+                "unit": "TFLOP/s",
+                "frac": round(achieved / (exp_peak if bound_alu else tensor_peak), 4),
+                "traffic": measured_traffic(dom_case.name),
+                "algorithmic_bytes": 2 * 4 * dom_case.B * dom_case.H * dom_case.N * dom_case.d
+                + 4 * dom_case.B * dom_case.H * dom_case.N,
+                "peak_source": ("derived: 16 ex2/clk/SM x 148 SMs x max SM clock x 4d FLOP per exp"
+                                if bound_alu else f"{peak_kind} bf16 matmul (burst)"),
+                "tensor_frac": round(achieved / tensor_peak, 4),
+                "tensor_peak": tensor_peak}
+        value = res["value"]
+        line = {"metric": METRIC, "value": round(value, 3), "unit": "TFLOPS", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(res["t_ms"] / args.steps, 5), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": wl.name, "description": wl.description,
+                           "cases": [c.name for c in run_cases], "per_gpu_batch": "one copy of every case",
+                           "l2": "flushed (512 MiB write) before every step",
+                           "parallelism": f"independent batches, {world} GPU(s)"},
+                "tensor_peak_frac": {"measured_bf16": round(value / world / tensor_peak, 4),
+                                     "datasheet_2250": round(value / world / 2250.0, 4)},
+                "cases": res["cases"], "roofline": roof, "clocks": res["clocks"],
+                "gpu_launches": args.steps * len(run_cases),
+                "kernel_source_hash": kernel_source_hash()}
+        if "e2e" in res:
+            line["e2e"] = res["e2e"]
+        if "suite" in res:
+            line["suite"] = res["suite"]
+        if world == 1 and not args.no_cpu:
+            line["cpu_baseline"] = cpu_baseline(run_cases)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
