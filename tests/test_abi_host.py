@@ -1,0 +1,64 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/fa.h declares, and rejects bad arguments before making
+any CUDA call."""
+
+from __future__ import annotations
+
+import ctypes
+import math
+
+import pytest
+
+from tiled_attention_12_b200 import binding as B
+
+
+def test_library_exports_every_declared_symbol():
+    names = B.declared_symbols()
+    assert {"fa_fwd", "fa_quantize_e4m3", "fa_fwd_fp8", "fa_last_device_status",
+            "fa_status_string", "fa_release"} <= set(names)
+    raw = ctypes.CDLL(B.LIB)
+    for n in names:
+        assert hasattr(raw, n), n
+
+
+def test_status_strings():
+    L = B.load()
+    for code in range(0, 7):
+        s = L.fa_status_string(code)
+        assert isinstance(s, bytes) and len(s) > 0
+    assert L.fa_status_string(0) == b"ok"
+    assert L.fa_status_string(99) == b"unknown status"
+
+
+P = 1 << 20          # a fake, 16-byte aligned pointer value; never dereferenced
+
+
+@pytest.mark.parametrize("args,expected", [
+    ((None, P, P, P * 2, None, 1, 1, 16, 64, 0.1, 0, 0), B.FA_ERR_INVALID),       # null q
+    ((P, P, P, P * 2, None, 0, 1, 16, 64, 0.1, 0, 0), B.FA_ERR_INVALID),          # B = 0
+    ((P, P, P, P * 2, None, 1, 1, 0, 64, 0.1, 0, 0), B.FA_ERR_INVALID),           # N = 0
+    ((P, P, P, P * 2, None, 1, 1, 16, 48, 0.1, 0, 0), B.FA_ERR_UNSUPPORTED),      # d = 48
+    ((P, P, P, P * 2, None, 1, 1, 16, 256, 0.1, 0, 0), B.FA_ERR_UNSUPPORTED),     # d = 256
+    ((P, P, P, P * 2, None, 1, 1, 16, 64, 0.1, 0, 2), B.FA_ERR_UNSUPPORTED),      # e4m3 needs d = 128
+    ((P, P, P, P * 2, None, 1, 1, 16, 64, 0.1, 0, 7), B.FA_ERR_INVALID),          # unknown dtype
+    ((P + 2, P, P, P * 2, None, 1, 1, 16, 64, 0.1, 0, 0), B.FA_ERR_INVALID),      # misaligned q
+    ((P, P, P, P * 2, P + 4, 1, 1, 16, 64, 0.1, 0, 0), B.FA_ERR_INVALID),         # misaligned lse
+    ((P, P, P, P * 2, None, 1, 1, 16, 64, 0.0, 0, 0), B.FA_ERR_INVALID),          # scale 0
+    ((P, P, P, P * 2, None, 1, 1, 16, 64, -1.0, 0, 0), B.FA_ERR_INVALID),         # scale < 0
+    ((P, P, P, P * 2, None, 1, 1, 16, 64, math.inf, 0, 0), B.FA_ERR_INVALID),     # scale inf
+    ((P, P, P, P * 2, None, 1, 1, 16, 64, math.nan, 0, 0), B.FA_ERR_INVALID),     # scale nan
+    ((P, P, P, P * 2, None, 1, 1, 16, 64, 0.1, 2, 0), B.FA_ERR_INVALID),          # causal = 2
+    ((P, P, P, P, None, 1, 1, 16, 64, 0.1, 0, 0), B.FA_ERR_INVALID),              # o aliases q
+    ((P, P, P, P * 2, None, 1 << 16, 1 << 16, 16, 64, 0.1, 0, 0), B.FA_ERR_INVALID),  # B*H overflow
+])
+def test_fwd_rejects_bad_arguments_without_cuda(args, expected):
+    assert B.load().fa_fwd(*args, None) == expected
+
+
+def test_other_entry_points_reject_bad_arguments():
+    L = B.load()
+    assert L.fa_quantize_e4m3(None, P, P, 1, 1, 16, 64, None) == B.FA_ERR_INVALID
+    assert L.fa_quantize_e4m3(P, P, P, 1, 1, 16, 40, None) == B.FA_ERR_UNSUPPORTED
+    assert L.fa_fwd_fp8(P, P, P, P, P, P * 2, None, 1, 1, 16, 64, 0.1, 0, None) == B.FA_ERR_UNSUPPORTED
+    assert L.fa_fwd_fp8(P, None, P, P, P, P * 2, None, 1, 1, 16, 128, 0.1, 0, None) == B.FA_ERR_INVALID
+    assert L.fa_fwd_fp8(P, P + 1, P, P, P, P * 2, None, 1, 1, 16, 128, 0.1, 0, None) == B.FA_ERR_INVALID
