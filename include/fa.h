@@ -51,7 +51,9 @@ typedef enum {
   FA_ERR_UNSUPPORTED = 2,  /* head dimension or dtype this build does not have */
   FA_ERR_ARCH = 3,         /* current device is not compute capability 10.x    */
   FA_ERR_CUDA = 4,         /* a CUDA runtime/driver call or launch failed      */
-  FA_ERR_TIMEOUT = 5       /* a kernel gave up on a bounded wait               */
+  FA_ERR_TIMEOUT = 5,      /* a kernel gave up on a bounded wait               */
+  FA_ERR_TOO_LARGE = 6     /* problem exceeds the fixed scratch of
+                              fa_fwd_e4m3_noalloc                               */
 } fa_status;
 
 typedef enum {
@@ -131,6 +133,46 @@ fa_status fa_debug_set_wait_limit(uint64_t nanoseconds);
  * Cleared after one launch.
  */
 fa_status fa_debug_withhold_arrival(int enable);
+
+/*
+ * fa_fwd_e4m3_noalloc — the FA_E4M3 forward without any allocation.
+ *
+ * No counterpart in the paper: this is a deployment variant of the FA_E4M3
+ * path of fa_fwd.  That path needs scratch for the quantised Q and K and
+ * grows it with cudaMalloc.  Some callers cannot allocate at all: code running
+ * inside a memory-pool or allocator callback (which must not re-enter the
+ * CUDA allocator), code on a device whose memory is already handed out in
+ * full to a pool it does not own, or a process whose policy forbids
+ * allocating after start-up.  This entry point keeps its scratch in one
+ * statically sized device array inside the library instead, and calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *
+ * Arguments, layout and results are those of fa_fwd with dtype = FA_E4M3:
+ * q, k, v bf16 [B, H, N, d], o bf16, lse fp32 [B, H, N] or NULL; d must be 128.
+ *
+ * Limits: B*H*N*d <= FA_NOALLOC_MAX_ELEMS (8 Mi elements per operand, e.g.
+ * B=1, H=16, N=4096) and B*H*ceil(N/128) <= FA_NOALLOC_MAX_TILES; larger
+ * problems return FA_ERR_TOO_LARGE without touching the device.  The array
+ * (FA_NOALLOC_SCRATCH_BYTES) is part of the library's device image: every
+ * GPU that loads the library holds it until the process exits.
+ *
+ * The first call on a device does a one-time set-up with that device
+ * current: it looks up the array's device address (cudaGetSymbolAddress) and
+ * clears its status word with a synchronous cudaMemset.  Make that first call
+ * before any stream capture.
+ *
+ * Every call on a device shares the one array, and the array keeps the last
+ * call's contents.  Calls whose work overlaps on the GPU (different streams,
+ * or different host threads without ordering) race on it; serialise them.
+ * A device-side wait that gives up is recorded in the array's own status
+ * word, not in the word fa_last_device_status reads.
+ */
+#define FA_NOALLOC_MAX_ELEMS (8u * 1024u * 1024u)
+#define FA_NOALLOC_MAX_TILES (65536u)
+#define FA_NOALLOC_SCRATCH_BYTES (2u * FA_NOALLOC_MAX_ELEMS + 2u * 4u * FA_NOALLOC_MAX_TILES + 256u)
+fa_status fa_fwd_e4m3_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                              int B, int H, int N, int d, float softmax_scale, int causal,
+                              void* stream);
 
 #ifdef __cplusplus
 }

@@ -14,7 +14,7 @@ import re
 
 from .build import INCLUDE, LIB
 
-FA_OK, FA_ERR_INVALID, FA_ERR_UNSUPPORTED, FA_ERR_ARCH, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(6)
+FA_OK, FA_ERR_INVALID, FA_ERR_UNSUPPORTED, FA_ERR_ARCH, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_TOO_LARGE = range(7)
 FA_BF16, FA_FP16, FA_E4M3 = 0, 1, 2
 
 _lib = None
@@ -46,13 +46,15 @@ def load():
     L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
     L.fa_quantize_e4m3.argtypes = [vp, vp, vp, i, i, i, i, vp]
     L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    L.fa_fwd_e4m3_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     L.fa_last_device_status.argtypes = [vp]
     L.fa_status_string.argtypes = [i]
     L.fa_status_string.restype = ctypes.c_char_p
     L.fa_release.argtypes = []
     L.fa_debug_set_wait_limit.argtypes = [ctypes.c_uint64]
     L.fa_debug_withhold_arrival.argtypes = [i]
-    for name in ("fa_fwd", "fa_quantize_e4m3", "fa_fwd_fp8", "fa_last_device_status", "fa_release",
+    for name in ("fa_fwd", "fa_quantize_e4m3", "fa_fwd_fp8", "fa_fwd_e4m3_noalloc", "fa_last_device_status",
+                 "fa_release",
                  "fa_debug_set_wait_limit", "fa_debug_withhold_arrival"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
@@ -143,6 +145,22 @@ def fa_fwd_fp8(q8, q_scale, k8, k_scale, v, o=None, lse=None, softmax_scale=None
     st = load().fa_fwd_fp8(_ptr(q8), _ptr(q_scale), _ptr(k8), _ptr(k_scale), _ptr(v), _ptr(o), _ptr(lse),
                            B, H, N, d, scale, int(bool(causal)), _stream(stream))
     _check(st, "fa_fwd_fp8")
+    return o, lse
+
+
+def fa_fwd_e4m3_noalloc(q, k, v, o, lse=None, softmax_scale=None, causal=False, stream=None):
+    """The e4m3 forward with library-static scratch: allocates nothing.
+
+    For callers that cannot allocate device memory (allocator callbacks,
+    fully pooled devices, no-allocation-after-start-up policies).  q, k, v
+    bf16 [B, H, N, 128]; o (and lse, if wanted) must be provided by the
+    caller.  Sizes beyond the fixed scratch raise FaError(FA_ERR_TOO_LARGE).
+    """
+    B, H, N, d = q.shape
+    scale = (1.0 / d ** 0.5) if softmax_scale is None else float(softmax_scale)
+    st = load().fa_fwd_e4m3_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, scale,
+                                    int(bool(causal)), _stream(stream))
+    _check(st, "fa_fwd_e4m3_noalloc")
     return o, lse
 
 

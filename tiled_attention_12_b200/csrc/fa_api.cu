@@ -253,6 +253,7 @@ const char* fa_status_string(fa_status status) {
     case FA_ERR_ARCH: return "device is not compute capability 10.x (sm_100)";
     case FA_ERR_CUDA: return "CUDA call or kernel launch failed";
     case FA_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
+    case FA_ERR_TOO_LARGE: return "problem exceeds the fixed scratch of fa_fwd_e4m3_noalloc";
     default: return "unknown status";
   }
 }

@@ -1,0 +1,167 @@
+// fa_noalloc.cu — fa_fwd_e4m3_noalloc: the e4m3 forward with its scratch in a
+// fixed, statically sized device array, for callers that cannot allocate.
+//
+// Who needs this: code that runs where cudaMalloc is off limits — inside a
+// host allocator callback or a custom memory pool that must not recurse into
+// the CUDA allocator, on a device whose memory is already fully handed out to
+// a pool owned by someone else, or in a process whose allocation policy
+// forbids allocations after start-up.  The regular FA_E4M3 path of fa_fwd
+// needs scratch for the quantised Q and K and grows it with cudaMalloc; this
+// variant uses the array below instead and calls no allocating routine.
+//
+// The array lives in the library's device image: every GPU that loads the
+// library holds it (FA_NOALLOC_SCRATCH_BYTES) until the process exits.
+//
+// Host code must not pass `g_noalloc_scratch` itself to a kernel: in host
+// code the name is a host-side stand-in, not a device address.  The device
+// address is looked up once per device with cudaGetSymbolAddress while that
+// device is current.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_fwd_kernel.cuh"
+#include "fa_launch.h"
+
+namespace {
+
+constexpr size_t kMaxElems = FA_NOALLOC_MAX_ELEMS;   // per operand (Q or K codes)
+constexpr size_t kMaxTiles = FA_NOALLOC_MAX_TILES;   // per operand (scales)
+constexpr size_t kCodesBytes = kMaxElems;            // one byte per e4m3 code
+constexpr size_t kScalesBytes = kMaxTiles * sizeof(float);
+constexpr size_t kStatusOffset = 2 * kCodesBytes + 2 * kScalesBytes;
+constexpr size_t kScratchBytes = kStatusOffset + 256;
+static_assert(kScratchBytes == FA_NOALLOC_SCRATCH_BYTES, "header and implementation disagree");
+
+// Layout: [q codes | k codes | q scales | k scales | status word (+pad)].
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct NoAllocDevice {
+  bool ready = false;
+  int sms = 0;
+  unsigned char* scratch = nullptr;  // device address of g_noalloc_scratch on this device
+};
+
+constexpr int kMaxDevices = 64;
+std::mutex g_na_mu;
+NoAllocDevice g_na[kMaxDevices];
+EncodeTiledFn g_na_encode = nullptr;
+
+// One-time set-up for the current device: architecture check, SM count, the
+// scratch array's device address and a cleared status word.
+fa_status noalloc_setup(NoAllocDevice** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_na_mu);
+  NoAllocDevice& s = g_na[dev];
+  if (!s.ready) {
+    int major = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return FA_ERR_CUDA;
+    if (major != 10) return FA_ERR_ARCH;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FA_ERR_CUDA;
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return FA_ERR_CUDA;
+    if (cudaMemset(static_cast<unsigned char*>(ptr) + kStatusOffset, 0, sizeof(unsigned int)) != cudaSuccess)
+      return FA_ERR_CUDA;
+    if (g_na_encode == nullptr) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return FA_ERR_CUDA;
+      g_na_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    s.sms = sms;
+    s.scratch = static_cast<unsigned char*>(ptr);
+    s.ready = true;
+  }
+  *out = &s;
+  return FA_OK;
+}
+
+// [BH, N, 128] tensor as a 3-D TMA map with a 128-byte swizzled box of 128
+// rows (the geometry the forward kernel's shared-memory layout expects).
+fa_status noalloc_map(CUtensorMap* map, const void* ptr, int BH, int N, bool codes) {
+  const int elem = codes ? 1 : 2;
+  const int row_bytes = 128 * elem;
+  cuuint64_t dims[3] = {128u, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(row_bytes) * N};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem), 128u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = g_na_encode(map, codes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                           const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_INVALID;
+}
+
+bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" fa_status fa_fwd_e4m3_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                                         int H, int N, int d, float softmax_scale, int causal, void* stream) {
+  if (B <= 0 || H <= 0 || N <= 0) return FA_ERR_INVALID;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o) return FA_ERR_INVALID;
+  if (!al16(q) || !al16(k) || !al16(v) || !al16(o) || (lse && !al16(lse))) return FA_ERR_INVALID;
+  if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.f) || (causal != 0 && causal != 1)) return FA_ERR_INVALID;
+  if (o == q || o == k || o == v) return FA_ERR_INVALID;
+  const long long BH = static_cast<long long>(B) * H;
+  const long long elems = BH * N * static_cast<long long>(d);
+  const long long tiles = BH * ((static_cast<long long>(N) + 127) / 128);
+  if (elems > static_cast<long long>(kMaxElems) || tiles > static_cast<long long>(kMaxTiles))
+    return FA_ERR_TOO_LARGE;
+
+  NoAllocDevice* dev = nullptr;
+  fa_status st = noalloc_setup(&dev);
+  if (st != FA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned char* q8 = dev->scratch;
+  unsigned char* k8 = dev->scratch + kCodesBytes;
+  float* qs = reinterpret_cast<float*>(dev->scratch + 2 * kCodesBytes);
+  float* ks = reinterpret_cast<float*>(dev->scratch + 2 * kCodesBytes + kScalesBytes);
+  unsigned int* status = reinterpret_cast<unsigned int*>(dev->scratch + kStatusOffset);
+
+  // The quantiser writes every code and scale the attention kernel reads, so
+  // nothing left over from an earlier call is ever consumed.
+  const int bh = static_cast<int>(BH);
+  if (fa::launch_quantize_e4m3(q, q8, qs, bh, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (fa::launch_quantize_e4m3(k, k8, ks, bh, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
+
+  fa::FwdLaunch l;
+  if ((st = noalloc_map(&l.map_q, q8, bh, N, true)) != FA_OK) return st;
+  if ((st = noalloc_map(&l.map_k, k8, bh, N, true)) != FA_OK) return st;
+  if ((st = noalloc_map(&l.map_v, v, bh, N, false)) != FA_OK) return st;
+  fa::FwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.o = o;
+  a.lse = lse;
+  a.q_scale = qs;
+  a.k_scale = ks;
+  a.status = status;
+  a.BH = bh;
+  a.N = N;
+  a.n_qpairs = (N + 255) / 256;
+  a.n_work = bh * a.n_qpairs;
+  a.n_qtiles = (N + 127) / 128;
+  a.causal = causal;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.wait_limit_ns = 2000000000ull;
+  a.withhold = 0;
+  l.grid = a.n_work < dev->sms ? a.n_work : dev->sms;
+  int g = (2 * l.grid + a.n_qpairs - 1) / a.n_qpairs;
+  a.group_heads = g < 1 ? 1 : (g > bh ? bh : g);
+  l.args = &a;
+  l.stream = s;
+  return fa::launch_fwd_e4m3(d, l) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
