@@ -91,9 +91,17 @@ struct FwdCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget exceeded");
   static constexpr int K_STEPS_QK = QK_ROW / 32;   // 32 bytes of K per S MMA (16 x 16-bit or 32 x 8-bit)
   static constexpr int K_STEPS_PV = BN / 16;       // 16 keys per P V MMA
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 384;  // 3 warpgroups
   static constexpr int MMA_WARP = 8;
-  static constexpr int LOAD_WARP = 9;
+  static constexpr int LOAD_WARP = 9;  // warps 10, 11 only rebalance registers
+  // Register split (setmaxnreg): the block launches with LAUNCH_REGS per
+  // thread; the two softmax warpgroups then take REG_SOFTMAX and the
+  // MMA/TMA warpgroup gives back down to REG_OTHER.  The shares must add up
+  // to exactly the launch total or setmaxnreg.inc would wait forever.
+  static constexpr int LAUNCH_REGS = 168;
+  static constexpr int REG_SOFTMAX = 216;
+  static constexpr int REG_OTHER = 72;
+  static_assert(2 * 128 * REG_SOFTMAX + 128 * REG_OTHER == THREADS * LAUNCH_REGS, "register split");
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t S_COL0 = 0, S_COL1 = 128, O_COL0 = 256, O_COL1 = 256 + D;
   static_assert(O_COL1 + D <= TMEM_COLS, "tensor memory budget exceeded");
@@ -160,8 +168,195 @@ __device__ __forceinline__ void record_failure(const FwdArgs& a, volatile int* a
   atomicOr(a.status, bit);
 }
 
+// ---------------------------------------------------------------- producer
+// One thread.  Per work tile: the Q tiles it needs, then K_j, V_j for every
+// K/V step into the ring.  Stage `it % NS` is reused in round `it / NS` once
+// the MMA thread has released round `it / NS - 1`.
 template <int D, int ELEM>
-__global__ void __launch_bounds__(320, 1)
+__device__ __noinline__ void producer_role(const FwdArgs& a, const Barriers& b, uint8_t* sQ, uint8_t* sKV,
+                                           const CUtensorMap* map_q, const CUtensorMap* map_k,
+                                           const CUtensorMap* map_v, volatile int* abort_flag) {
+  using C = FwdCfg<D, ELEM>;
+  const uint64_t limit = a.wait_limit_ns;
+  tma_prefetch_desc(map_q);
+  tma_prefetch_desc(map_k);
+  tma_prefetch_desc(map_v);
+  int kv_it = 0, q_use0 = 0, q_use1 = 0;
+  bool withhold = a.withhold != 0;
+  bool ok = true;
+  for (int w = blockIdx.x; ok && w < a.n_work; w += gridDim.x) {
+    const WorkTile t = decode_work(a, w);
+    const int q0 = t.tp * 256;
+    const int n0 = kv_tiles(a, q0), n1 = kv_tiles(a, q0 + 128);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int n = i ? n1 : n0;
+      int& use = i ? q_use1 : q_use0;
+      if (n == 0) continue;
+      if (use > 0 && !wait_bounded(&b.q_empty[i], (use - 1) & 1, abort_flag, limit)) {
+        ok = false;
+        break;
+      }
+      mbar_arrive_expect_tx(&b.q_full[i], C::Q_TILE);
+#pragma unroll
+      for (int c = 0; c < C::QK_ROW / C::SW_QK; ++c)
+        tma_load_3d(sQ + i * C::Q_TILE + c * C::BM * C::SW_QK, map_q, &b.q_full[i], c * (C::SW_QK / C::QK_BYTES),
+                    q0 + i * 128, t.bh);
+      ++use;
+    }
+    const int nkv = n0 > n1 ? n0 : n1;
+    for (int j = 0; ok && j < nkv; ++j) {
+#pragma unroll
+      for (int kind = 0; kind < 2; ++kind) {
+        const int s = kv_it % C::NS;
+        const int r = kv_it / C::NS;
+        if (r > 0 && !wait_bounded(&b.kv_empty[s], (r - 1) & 1, abort_flag, limit)) {
+          ok = false;
+          break;
+        }
+        ++kv_it;
+        if (withhold && kv_it == 1) continue;  // test hook: this tile never arrives
+        uint8_t* dst = sKV + s * C::STAGE;
+        if (kind == 0) {
+          mbar_arrive_expect_tx(&b.kv_full[s], C::K_TILE);
+#pragma unroll
+          for (int c = 0; c < C::QK_ROW / C::SW_QK; ++c)
+            tma_load_3d(dst + c * C::BN * C::SW_QK, map_k, &b.kv_full[s], c * (C::SW_QK / C::QK_BYTES), j * 128,
+                        t.bh);
+        } else {
+          mbar_arrive_expect_tx(&b.kv_full[s], C::V_TILE);
+#pragma unroll
+          for (int c = 0; c < C::V_ROW / C::SW_V; ++c)
+            tma_load_3d(dst + c * C::BN * C::SW_V, map_v, &b.kv_full[s], c * (C::SW_V / 2), j * 128, t.bh);
+        }
+      }
+    }
+  }
+  if (!ok) record_failure(a, abort_flag, kStatusProducer);
+  // Drain: every bulk copy issued has landed before the CTA may exit (after
+  // a normal run these phases are long complete).  The last NS ring indices
+  // are the only ones that can still be in flight.
+  volatile int never = 0;
+  bool drained = true;
+  if (q_use0 > 0) drained &= wait_bounded(&b.q_full[0], (q_use0 - 1) & 1, &never, limit);
+  if (q_use1 > 0) drained &= wait_bounded(&b.q_full[1], (q_use1 - 1) & 1, &never, limit);
+  for (int idx = kv_it - 1; idx >= 0 && idx >= kv_it - C::NS; --idx) {
+    if (withhold && idx == 0) continue;
+    drained &= wait_bounded(&b.kv_full[idx % C::NS], (idx / C::NS) & 1, &never, limit);
+  }
+  if (!drained) atomicOr(a.status, kStatusDrain);
+}
+
+// ---------------------------------------------------------------- MMA
+// One thread issues every tcgen05.mma.  Descriptors are built once per
+// operand base and advanced by adding (byte offset >> 4) to the start-address
+// field, which cannot overflow for shared-memory addresses below 256 KB.
+template <int D, int ELEM>
+__device__ __noinline__ void mma_role(const FwdArgs& a, const Barriers& b, uint32_t sQ_addr, uint32_t sKV_addr,
+                                      uint32_t tmem, volatile int* abort_flag) {
+  using C = FwdCfg<D, ELEM>;
+  const uint64_t limit = a.wait_limit_ns;
+  const uint64_t dq0 = smem_desc(sQ_addr, 16, 8 * C::SW_QK, C::SWZ_QK);
+  const uint64_t dkv0 = smem_desc(sKV_addr, 16, 8 * C::SW_QK, C::SWZ_QK);
+  const uint64_t dv0 = smem_desc(sKV_addr, C::BN * C::SW_V, 8 * C::SW_V, C::SWZ_V);
+  int kv_it = 0, q_use0 = 0, q_use1 = 0, p_cnt0 = 0, p_cnt1 = 0;
+
+  auto issue_s = [&](int i, int stage) {
+    const uint32_t d_tmem = tmem + (i ? C::S_COL1 : C::S_COL0);
+    const uint64_t qa = dq0 + ((i * C::Q_TILE) >> 4);
+    const uint64_t ka = dkv0 + ((stage * C::STAGE) >> 4);
+#pragma unroll
+    for (int kk = 0; kk < C::K_STEPS_QK; ++kk) {
+      const uint32_t off = ((kk * 32) / C::SW_QK) * (C::BM * C::SW_QK) + ((kk * 32) % C::SW_QK);
+      if constexpr (ELEM == kElemE4M3)
+        mma_f8_ss(d_tmem, qa + (off >> 4), ka + (off >> 4), C::IDESC_QK, kk > 0);
+      else
+        mma_f16_ss(d_tmem, qa + (off >> 4), ka + (off >> 4), C::IDESC_QK, kk > 0);
+    }
+  };
+  auto issue_pv = [&](int i, int stage, bool accumulate) {
+    const uint32_t d_tmem = tmem + (i ? C::O_COL1 : C::O_COL0);
+    const uint32_t p_tmem = tmem + (i ? C::S_COL1 : C::S_COL0);
+    const uint64_t va = dv0 + ((stage * C::STAGE) >> 4);
+#pragma unroll
+    for (int kk = 0; kk < C::K_STEPS_PV; ++kk)
+      mma_f16_ts(d_tmem, p_tmem + kk * 8, va + ((kk * 16 * C::SW_V) >> 4), C::IDESC_PV,
+                 (accumulate || kk > 0) ? 1u : 0u);
+  };
+
+  bool ok = true;
+  for (int w = blockIdx.x; ok && w < a.n_work; w += gridDim.x) {
+    const WorkTile t = decode_work(a, w);
+    const int q0 = t.tp * 256;
+    const int n0 = kv_tiles(a, q0), n1 = kv_tiles(a, q0 + 128);
+    const int nkv = n0 > n1 ? n0 : n1;
+    if (n0 > 0 && !wait_bounded(&b.q_full[0], (q_use0++) & 1, abort_flag, limit)) { ok = false; break; }
+    if (n1 > 0 && !wait_bounded(&b.q_full[1], (q_use1++) & 1, abort_flag, limit)) { ok = false; break; }
+    int sk = kv_it % C::NS;
+    if (!wait_bounded(&b.kv_full[sk], (kv_it / C::NS) & 1, abort_flag, limit)) { ok = false; break; }
+    ++kv_it;
+    tc_fence_after();
+    if (n0 > 0) {
+      issue_s(0, sk);
+      tc_commit(&b.s_full[0]);
+      if (n0 == 1) tc_commit(&b.q_empty[0]);
+    }
+    if (n1 > 0) {
+      issue_s(1, sk);
+      tc_commit(&b.s_full[1]);
+      if (n1 == 1) tc_commit(&b.q_empty[1]);
+    }
+    tc_commit(&b.kv_empty[sk]);
+    for (int j = 0; j < nkv; ++j) {
+      const int sv = kv_it % C::NS;
+      if (!wait_bounded(&b.kv_full[sv], (kv_it / C::NS) & 1, abort_flag, limit)) { ok = false; break; }
+      ++kv_it;
+      tc_fence_after();
+      if (j < n0) {
+        if (!wait_bounded(&b.p_full[0], (p_cnt0++) & 1, abort_flag, limit)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(0, sv, j > 0);
+        if (j == n0 - 1) tc_commit(&b.o_full[0]);
+      }
+      const bool next = j + 1 < nkv;
+      int sk2 = 0;
+      if (next) {
+        sk2 = kv_it % C::NS;
+        if (!wait_bounded(&b.kv_full[sk2], (kv_it / C::NS) & 1, abort_flag, limit)) { ok = false; break; }
+        ++kv_it;
+        tc_fence_after();
+        if (j + 1 < n0) {
+          issue_s(0, sk2);
+          tc_commit(&b.s_full[0]);
+          if (j + 1 == n0 - 1) tc_commit(&b.q_empty[0]);
+        }
+      }
+      if (j < n1) {
+        if (!wait_bounded(&b.p_full[1], (p_cnt1++) & 1, abort_flag, limit)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(1, sv, j > 0);
+        if (j == n1 - 1) tc_commit(&b.o_full[1]);
+      }
+      tc_commit(&b.kv_empty[sv]);
+      if (next) {
+        if (j + 1 < n1) {
+          issue_s(1, sk2);
+          tc_commit(&b.s_full[1]);
+          if (j + 1 == n1 - 1) tc_commit(&b.q_empty[1]);
+        }
+        tc_commit(&b.kv_empty[sk2]);
+      }
+    }
+  }
+  if (!ok) record_failure(a, abort_flag, kStatusMma);
+  // Drain: all issued MMAs complete before tensor memory is released.
+  tc_commit(b.mma_done);
+  volatile int never = 0;
+  if (!wait_bounded(b.mma_done, 0, &never, limit)) atomicOr(a.status, kStatusDrain);
+}
+
+template <int D, int ELEM>
+__global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                   const __grid_constant__ CUtensorMap map_v, const FwdArgs a) {
   using C = FwdCfg<D, ELEM>;
@@ -214,195 +409,17 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = tmem_holder;
   const uint64_t limit = a.wait_limit_ns;
 
-  if (warp == C::LOAD_WARP) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      tma_prefetch_desc(&map_q);
-      tma_prefetch_desc(&map_k);
-      tma_prefetch_desc(&map_v);
-      int kv_it = 0;
-      int q_use[2] = {0, 0};
-      int last_round[C::NS];
-#pragma unroll
-      for (int s = 0; s < C::NS; ++s) last_round[s] = -1;
-      bool withhold = a.withhold != 0;
-      auto run = [&]() -> bool {
-        for (int w = blockIdx.x; w < a.n_work; w += gridDim.x) {
-          const WorkTile t = decode_work(a, w);
-          const int q0 = t.tp * 256;
-          const int n[2] = {kv_tiles(a, q0), kv_tiles(a, q0 + 128)};
-          for (int i = 0; i < 2; ++i) {
-            if (n[i] == 0) continue;
-            if (q_use[i] > 0 && !wait_bounded(&b.q_empty[i], (q_use[i] - 1) & 1, abort_flag, limit))
-              return false;
-            mbar_arrive_expect_tx(&b.q_full[i], C::Q_TILE);
-#pragma unroll
-            for (int c = 0; c < C::QK_ROW / C::SW_QK; ++c)
-              tma_load_3d(sQ + i * C::Q_TILE + c * C::BM * C::SW_QK, &map_q, &b.q_full[i],
-                          c * (C::SW_QK / C::QK_BYTES), q0 + i * 128, t.bh);
-            ++q_use[i];
-          }
-          const int nkv = n[0] > n[1] ? n[0] : n[1];
-          for (int j = 0; j < nkv; ++j) {
-#pragma unroll
-            for (int kind = 0; kind < 2; ++kind) {
-              const int s = kv_it % C::NS;
-              const int r = kv_it / C::NS;
-              if (r > 0 && !wait_bounded(&b.kv_empty[s], (r - 1) & 1, abort_flag, limit)) return false;
-              ++kv_it;
-              if (withhold) {  // test hook: this tile never arrives
-                withhold = false;
-                continue;
-              }
-              uint8_t* dst = sKV + s * C::STAGE;
-              if (kind == 0) {
-                mbar_arrive_expect_tx(&b.kv_full[s], C::K_TILE);
-#pragma unroll
-                for (int c = 0; c < C::QK_ROW / C::SW_QK; ++c)
-                  tma_load_3d(dst + c * C::BN * C::SW_QK, &map_k, &b.kv_full[s], c * (C::SW_QK / C::QK_BYTES),
-                              j * 128, t.bh);
-              } else {
-                mbar_arrive_expect_tx(&b.kv_full[s], C::V_TILE);
-#pragma unroll
-                for (int c = 0; c < C::V_ROW / C::SW_V; ++c)
-                  tma_load_3d(dst + c * C::BN * C::SW_V, &map_v, &b.kv_full[s], c * (C::SW_V / 2), j * 128, t.bh);
-              }
-              last_round[s] = r;
-            }
-          }
-        }
-        return true;
-      };
-      if (!run()) record_failure(a, abort_flag, kStatusProducer);
-      // Drain: every bulk copy this thread issued has landed before the CTA
-      // may exit (normal completion finds these phases already complete).
-      volatile int never = 0;
-      bool drained = true;
-      for (int i = 0; i < 2; ++i)
-        if (q_use[i] > 0) drained &= wait_bounded(&b.q_full[i], (q_use[i] - 1) & 1, &never, limit);
-#pragma unroll
-      for (int s = 0; s < C::NS; ++s)
-        if (last_round[s] >= 0) drained &= wait_bounded(&b.kv_full[s], last_round[s] & 1, &never, limit);
-      if (!drained) atomicOr(a.status, kStatusDrain);
-    }
-  } else if (warp == C::MMA_WARP) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t sQ_addr = smem_u32(sQ);
-      const uint32_t sKV_addr = smem_u32(sKV);
-      int kv_it = 0;
-      int q_use[2] = {0, 0};
-      int p_cnt[2] = {0, 0};
-
-      auto issue_s = [&](int i, int stage) {
-        const uint32_t d_tmem = tmem + (i ? C::S_COL1 : C::S_COL0);
-        const uint32_t qa = sQ_addr + i * C::Q_TILE;
-        const uint32_t ka = sKV_addr + stage * C::STAGE;
-#pragma unroll
-        for (int kk = 0; kk < C::K_STEPS_QK; ++kk) {
-          const uint32_t byte = kk * 32;
-          const uint32_t off = (byte / C::SW_QK) * (C::BM * C::SW_QK) + (byte % C::SW_QK);
-          const uint64_t ad = smem_desc(qa + off, 16, 8 * C::SW_QK, C::SWZ_QK);
-          const uint64_t bd = smem_desc(ka + off, 16, 8 * C::SW_QK, C::SWZ_QK);
-          if constexpr (ELEM == kElemE4M3)
-            mma_f8_ss(d_tmem, ad, bd, C::IDESC_QK, kk > 0);
-          else
-            mma_f16_ss(d_tmem, ad, bd, C::IDESC_QK, kk > 0);
-        }
-      };
-      auto issue_pv = [&](int i, int stage, bool accumulate) {
-        const uint32_t d_tmem = tmem + (i ? C::O_COL1 : C::O_COL0);
-        const uint32_t p_tmem = tmem + (i ? C::S_COL1 : C::S_COL0);
-        const uint32_t va = sKV_addr + stage * C::STAGE;
-#pragma unroll
-        for (int kk = 0; kk < C::K_STEPS_PV; ++kk) {
-          const uint64_t bd = smem_desc(va + kk * 16 * C::SW_V, C::BN * C::SW_V, 8 * C::SW_V, C::SWZ_V);
-          mma_f16_ts(d_tmem, p_tmem + kk * 8, bd, C::IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
-        }
-      };
-      auto acquire = [&](int& stage) -> bool {
-        stage = kv_it % C::NS;
-        const int r = kv_it / C::NS;
-        ++kv_it;
-        if (!wait_bounded(&b.kv_full[stage], r & 1, abort_flag, limit)) return false;
-        tc_fence_after();
-        return true;
-      };
-
-      auto run = [&]() -> bool {
-        for (int w = blockIdx.x; w < a.n_work; w += gridDim.x) {
-          const WorkTile t = decode_work(a, w);
-          const int q0 = t.tp * 256;
-          const int n0 = kv_tiles(a, q0), n1 = kv_tiles(a, q0 + 128);
-          const int nkv = n0 > n1 ? n0 : n1;
-          if (n0 > 0) {
-            if (!wait_bounded(&b.q_full[0], q_use[0] & 1, abort_flag, limit)) return false;
-            ++q_use[0];
-          }
-          if (n1 > 0) {
-            if (!wait_bounded(&b.q_full[1], q_use[1] & 1, abort_flag, limit)) return false;
-            ++q_use[1];
-          }
-          int sk;
-          if (!acquire(sk)) return false;
-          if (n0 > 0) {
-            issue_s(0, sk);
-            tc_commit(&b.s_full[0]);
-            if (n0 == 1) tc_commit(&b.q_empty[0]);
-          }
-          if (n1 > 0) {
-            issue_s(1, sk);
-            tc_commit(&b.s_full[1]);
-            if (n1 == 1) tc_commit(&b.q_empty[1]);
-          }
-          tc_commit(&b.kv_empty[sk]);
-          for (int j = 0; j < nkv; ++j) {
-            int sv;
-            if (!acquire(sv)) return false;
-            if (j < n0) {
-              if (!wait_bounded(&b.p_full[0], p_cnt[0] & 1, abort_flag, limit)) return false;
-              ++p_cnt[0];
-              tc_fence_after();
-              issue_pv(0, sv, j > 0);
-              if (j == n0 - 1) tc_commit(&b.o_full[0]);
-            }
-            const bool next = j + 1 < nkv;
-            int sk2 = 0;
-            if (next) {
-              if (!acquire(sk2)) return false;
-              if (j + 1 < n0) {
-                issue_s(0, sk2);
-                tc_commit(&b.s_full[0]);
-                if (j + 1 == n0 - 1) tc_commit(&b.q_empty[0]);
-              }
-            }
-            if (j < n1) {
-              if (!wait_bounded(&b.p_full[1], p_cnt[1] & 1, abort_flag, limit)) return false;
-              ++p_cnt[1];
-              tc_fence_after();
-              issue_pv(1, sv, j > 0);
-              if (j == n1 - 1) tc_commit(&b.o_full[1]);
-            }
-            tc_commit(&b.kv_empty[sv]);
-            if (next) {
-              if (j + 1 < n1) {
-                issue_s(1, sk2);
-                tc_commit(&b.s_full[1]);
-                if (j + 1 == n1 - 1) tc_commit(&b.q_empty[1]);
-              }
-              tc_commit(&b.kv_empty[sk2]);
-            }
-          }
-        }
-        return true;
-      };
-      if (!run()) record_failure(a, abort_flag, kStatusMma);
-      // Drain: all issued MMAs complete before tensor memory is released.
-      tc_commit(b.mma_done);
-      volatile int never = 0;
-      if (!wait_bounded(b.mma_done, 0, &never, limit)) atomicOr(a.status, kStatusDrain);
-    }
+  // Each role's code sits inside the branch that set its register budget, so
+  // the compiler allocates the softmax code for REG_SOFTMAX registers.
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(C::REG_OTHER));
+    if (warp == C::LOAD_WARP && lane == 0)
+      producer_role<D, ELEM>(a, b, sQ, sKV, &map_q, &map_k, &map_v, abort_flag);
+    else if (warp == C::MMA_WARP && lane == 0)
+      mma_role<D, ELEM>(a, b, smem_u32(sQ), smem_u32(sKV), tmem, abort_flag);
+    // warps 10 and 11 only give their registers away
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(C::REG_SOFTMAX));
     // ------------------------------------------------------------ softmax
     const int wg = warp >> 2;            // which Q tile
     const int wq = warp & 3;             // warp within the warpgroup -> TMEM lanes
