@@ -31,3 +31,16 @@ int fwd_smem_bytes(int d, int elem) {
 }
 
 }  // namespace fa
+
+#ifdef FA_TRACE
+// Trace-enabled builds only: copies the trace array (8 slices of
+// FA_TRACE_CAP / 8 records; unused records are 0) out and clears it.
+extern "C" int fa_trace_read(unsigned long long* host, int cap) {
+  if (cap < FA_TRACE_CAP) return -1;
+  if (cudaMemcpyFromSymbol(host, fa::g_fa_trace, FA_TRACE_CAP * sizeof(unsigned long long)) != cudaSuccess)
+    return -1;
+  static unsigned long long zeros[FA_TRACE_CAP];
+  if (cudaMemcpyToSymbol(fa::g_fa_trace, zeros, sizeof(zeros)) != cudaSuccess) return -1;
+  return FA_TRACE_CAP;
+}
+#endif

@@ -39,6 +39,14 @@
 
 #include "ptx.cuh"
 
+#ifndef FA_POLY_MASK
+#define FA_POLY_MASK 0x4924u
+#endif
+// shared-memory bytes for the Q tiles plus the K/V ring (sets the ring depth)
+#ifndef FA_SMEM_FOR_TILES
+#define FA_SMEM_FOR_TILES (200 * 1024)
+#endif
+
 namespace fa {
 
 enum : int { kElemBF16 = 0, kElemF16 = 1, kElemE4M3 = 2 };
@@ -79,11 +87,11 @@ struct FwdCfg {
   static constexpr int K_TILE = BN * QK_ROW;
   static constexpr int V_TILE = BN * V_ROW;
   static constexpr int STAGE = K_TILE > V_TILE ? K_TILE : V_TILE;
-  static constexpr int NS_FIT = (200 * 1024 - 2 * Q_TILE) / STAGE;
+  static constexpr int NS_FIT = (FA_SMEM_FOR_TILES - 2 * Q_TILE) / STAGE;
   static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;  // K/V ring depth
   static_assert(NS >= 2, "ring too shallow");
   static constexpr int TILE_BYTES = 2 * Q_TILE + NS * STAGE;
-  static constexpr int NUM_BARS = 2 + 2 + 2 * NS + 2 + 2 + 2 + 1;
+  static constexpr int NUM_BARS = 13 + 2 * NS;
   // at least 120 KB so that two CTAs never share an SM (each holds all 512
   // tensor-memory columns; a second resident CTA would only wait)
   static constexpr int SMEM_NEED = 1024 + TILE_BYTES + 8 * NUM_BARS;
@@ -99,8 +107,8 @@ struct FwdCfg {
   // MMA/TMA warpgroup gives back down to REG_OTHER.  The shares must add up
   // to exactly the launch total or setmaxnreg.inc would wait forever.
   static constexpr int LAUNCH_REGS = 168;
-  static constexpr int REG_SOFTMAX = 216;
-  static constexpr int REG_OTHER = 72;
+  static constexpr int REG_SOFTMAX = 208;
+  static constexpr int REG_OTHER = 88;
   static_assert(2 * 128 * REG_SOFTMAX + 128 * REG_OTHER == THREADS * LAUNCH_REGS, "register split");
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t S_COL0 = 0, S_COL1 = 128, O_COL0 = 256, O_COL1 = 256 + D;
@@ -112,17 +120,31 @@ struct FwdCfg {
   static constexpr uint32_t SWZ_QK = SW_QK == 128 ? 2u : 4u;
   static constexpr uint32_t SWZ_V = SW_V == 128 ? 2u : 4u;
   static constexpr float TAU = 8.0f;  // deferred-rescale threshold (log2 units)
+  // Column pairs (of every 16) whose exponentials use the FMA-pipe
+  // polynomial instead of the special-function unit: 5 of 16 pairs.
+  static constexpr uint32_t POLY_MASK = FA_POLY_MASK;
 };
 
-struct Barriers {
-  uint64_t* q_full;    // [2]  TMA -> MMA
-  uint64_t* q_empty;   // [2]  MMA -> TMA
-  uint64_t* kv_full;   // [NS] TMA -> MMA
-  uint64_t* kv_empty;  // [NS] MMA -> TMA
-  uint64_t* s_full;    // [2]  MMA -> softmax i
-  uint64_t* p_full;    // [2]  softmax i -> MMA (4 warp arrivals)
-  uint64_t* o_full;    // [2]  MMA -> softmax i (epilogue)
-  uint64_t* mma_done;  // [1]  MMA drain
+// Barrier slots (8 bytes each) after the tiles in shared memory, addressed by
+// their 32-bit shared-memory address.
+template <int NS>
+struct Bars {
+  uint32_t base;
+  __device__ __forceinline__ uint32_t q_full(int i) const { return base + 8u * i; }          // TMA -> MMA
+  __device__ __forceinline__ uint32_t q_empty(int i) const { return base + 8u * (2 + i); }   // MMA -> TMA
+  __device__ __forceinline__ uint32_t kv_full(int s) const { return base + 8u * (4 + s); }   // TMA -> MMA
+  __device__ __forceinline__ uint32_t kv_empty(int s) const { return base + 8u * (4 + NS + s); }  // MMA -> TMA
+  __device__ __forceinline__ uint32_t s_full(int i) const { return base + 8u * (4 + 2 * NS + i); }  // MMA -> softmax i
+  // softmax i -> MMA, one barrier per half of P (4 warp arrivals each).  Two
+  // barriers rather than two phases of one: the softmax may finish both
+  // halves before the MMA thread looks, and a parity wait cannot tell phase k
+  // from phase k + 2.
+  __device__ __forceinline__ uint32_t p_full(int i, int half) const {
+    return base + 8u * (6 + 2 * NS + 2 * i + half);
+  }
+  __device__ __forceinline__ uint32_t o_full(int i) const { return base + 8u * (10 + 2 * NS + i); }  // MMA -> epilogue
+  __device__ __forceinline__ uint32_t mma_done() const { return base + 8u * (12 + 2 * NS); }
+  static constexpr int COUNT = 13 + 2 * NS;
 };
 
 struct WorkTile {
@@ -173,16 +195,17 @@ __device__ __forceinline__ void record_failure(const FwdArgs& a, volatile int* a
 // K/V step into the ring.  Stage `it % NS` is reused in round `it / NS` once
 // the MMA thread has released round `it / NS - 1`.
 template <int D, int ELEM>
-__device__ __noinline__ void producer_role(const FwdArgs& a, const Barriers& b, uint8_t* sQ, uint8_t* sKV,
-                                           const CUtensorMap* map_q, const CUtensorMap* map_k,
-                                           const CUtensorMap* map_v, volatile int* abort_flag) {
+__device__ __forceinline__ void producer_role(const FwdArgs& a, const Bars<FwdCfg<D, ELEM>::NS> b, uint32_t sQ,
+                                              uint32_t sKV, const CUtensorMap* map_q, const CUtensorMap* map_k,
+                                              const CUtensorMap* map_v, volatile int* abort_flag) {
   using C = FwdCfg<D, ELEM>;
   const uint64_t limit = a.wait_limit_ns;
   tma_prefetch_desc(map_q);
   tma_prefetch_desc(map_k);
   tma_prefetch_desc(map_v);
   int kv_it = 0, q_use0 = 0, q_use1 = 0;
-  bool withhold = a.withhold != 0;
+  FA_TRACE_DECL;
+  const bool withhold = a.withhold != 0;
   bool ok = true;
   for (int w = blockIdx.x; ok && w < a.n_work; w += gridDim.x) {
     const WorkTile t = decode_work(a, w);
@@ -193,14 +216,14 @@ __device__ __noinline__ void producer_role(const FwdArgs& a, const Barriers& b, 
       const int n = i ? n1 : n0;
       int& use = i ? q_use1 : q_use0;
       if (n == 0) continue;
-      if (use > 0 && !wait_bounded(&b.q_empty[i], (use - 1) & 1, abort_flag, limit)) {
+      if (use > 0 && !wait_bounded(b.q_empty(i), (use - 1) & 1, abort_flag, limit)) {
         ok = false;
         break;
       }
-      mbar_arrive_expect_tx(&b.q_full[i], C::Q_TILE);
+      mbar_arrive_expect_tx(b.q_full(i), C::Q_TILE);
 #pragma unroll
       for (int c = 0; c < C::QK_ROW / C::SW_QK; ++c)
-        tma_load_3d(sQ + i * C::Q_TILE + c * C::BM * C::SW_QK, map_q, &b.q_full[i], c * (C::SW_QK / C::QK_BYTES),
+        tma_load_3d(sQ + i * C::Q_TILE + c * C::BM * C::SW_QK, map_q, b.q_full(i), c * (C::SW_QK / C::QK_BYTES),
                     q0 + i * 128, t.bh);
       ++use;
     }
@@ -210,24 +233,26 @@ __device__ __noinline__ void producer_role(const FwdArgs& a, const Barriers& b, 
       for (int kind = 0; kind < 2; ++kind) {
         const int s = kv_it % C::NS;
         const int r = kv_it / C::NS;
-        if (r > 0 && !wait_bounded(&b.kv_empty[s], (r - 1) & 1, abort_flag, limit)) {
+        FA_TRACE_EV(3, 50 + kind, j);
+        if (r > 0 && !wait_bounded(b.kv_empty(s), (r - 1) & 1, abort_flag, limit)) {
           ok = false;
           break;
         }
+        FA_TRACE_EV(3, 52 + kind, j);
         ++kv_it;
         if (withhold && kv_it == 1) continue;  // test hook: this tile never arrives
-        uint8_t* dst = sKV + s * C::STAGE;
+        const uint32_t dst = sKV + s * C::STAGE;
         if (kind == 0) {
-          mbar_arrive_expect_tx(&b.kv_full[s], C::K_TILE);
+          mbar_arrive_expect_tx(b.kv_full(s), C::K_TILE);
 #pragma unroll
           for (int c = 0; c < C::QK_ROW / C::SW_QK; ++c)
-            tma_load_3d(dst + c * C::BN * C::SW_QK, map_k, &b.kv_full[s], c * (C::SW_QK / C::QK_BYTES), j * 128,
+            tma_load_3d(dst + c * C::BN * C::SW_QK, map_k, b.kv_full(s), c * (C::SW_QK / C::QK_BYTES), j * 128,
                         t.bh);
         } else {
-          mbar_arrive_expect_tx(&b.kv_full[s], C::V_TILE);
+          mbar_arrive_expect_tx(b.kv_full(s), C::V_TILE);
 #pragma unroll
           for (int c = 0; c < C::V_ROW / C::SW_V; ++c)
-            tma_load_3d(dst + c * C::BN * C::SW_V, map_v, &b.kv_full[s], c * (C::SW_V / 2), j * 128, t.bh);
+            tma_load_3d(dst + c * C::BN * C::SW_V, map_v, b.kv_full(s), c * (C::SW_V / 2), j * 128, t.bh);
         }
       }
     }
@@ -238,11 +263,11 @@ __device__ __noinline__ void producer_role(const FwdArgs& a, const Barriers& b, 
   // are the only ones that can still be in flight.
   volatile int never = 0;
   bool drained = true;
-  if (q_use0 > 0) drained &= wait_bounded(&b.q_full[0], (q_use0 - 1) & 1, &never, limit);
-  if (q_use1 > 0) drained &= wait_bounded(&b.q_full[1], (q_use1 - 1) & 1, &never, limit);
+  if (q_use0 > 0) drained &= wait_bounded(b.q_full(0), (q_use0 - 1) & 1, &never, limit);
+  if (q_use1 > 0) drained &= wait_bounded(b.q_full(1), (q_use1 - 1) & 1, &never, limit);
   for (int idx = kv_it - 1; idx >= 0 && idx >= kv_it - C::NS; --idx) {
     if (withhold && idx == 0) continue;
-    drained &= wait_bounded(&b.kv_full[idx % C::NS], (idx / C::NS) & 1, &never, limit);
+    drained &= wait_bounded(b.kv_full(idx % C::NS), (idx / C::NS) & 1, &never, limit);
   }
   if (!drained) atomicOr(a.status, kStatusDrain);
 }
@@ -252,14 +277,15 @@ __device__ __noinline__ void producer_role(const FwdArgs& a, const Barriers& b, 
 // operand base and advanced by adding (byte offset >> 4) to the start-address
 // field, which cannot overflow for shared-memory addresses below 256 KB.
 template <int D, int ELEM>
-__device__ __noinline__ void mma_role(const FwdArgs& a, const Barriers& b, uint32_t sQ_addr, uint32_t sKV_addr,
-                                      uint32_t tmem, volatile int* abort_flag) {
+__device__ __forceinline__ void mma_role(const FwdArgs& a, const Bars<FwdCfg<D, ELEM>::NS> b, uint32_t sQ_addr,
+                                         uint32_t sKV_addr, uint32_t tmem, volatile int* abort_flag) {
   using C = FwdCfg<D, ELEM>;
   const uint64_t limit = a.wait_limit_ns;
   const uint64_t dq0 = smem_desc(sQ_addr, 16, 8 * C::SW_QK, C::SWZ_QK);
   const uint64_t dkv0 = smem_desc(sKV_addr, 16, 8 * C::SW_QK, C::SWZ_QK);
   const uint64_t dv0 = smem_desc(sKV_addr, C::BN * C::SW_V, 8 * C::SW_V, C::SWZ_V);
   int kv_it = 0, q_use0 = 0, q_use1 = 0, p_cnt0 = 0, p_cnt1 = 0;
+  FA_TRACE_DECL;
 
   auto issue_s = [&](int i, int stage) {
     const uint32_t d_tmem = tmem + (i ? C::S_COL1 : C::S_COL0);
@@ -274,14 +300,29 @@ __device__ __noinline__ void mma_role(const FwdArgs& a, const Barriers& b, uint3
         mma_f16_ss(d_tmem, qa + (off >> 4), ka + (off >> 4), C::IDESC_QK, kk > 0);
     }
   };
-  auto issue_pv = [&](int i, int stage, bool accumulate) {
+  // O_i += P_i V over keys [64*half, 64*half + 64) of the K/V tile.
+  auto issue_pv_half = [&](int i, int stage, int half, bool accumulate) {
     const uint32_t d_tmem = tmem + (i ? C::O_COL1 : C::O_COL0);
     const uint32_t p_tmem = tmem + (i ? C::S_COL1 : C::S_COL0);
     const uint64_t va = dv0 + ((stage * C::STAGE) >> 4);
 #pragma unroll
-    for (int kk = 0; kk < C::K_STEPS_PV; ++kk)
+    for (int k = 0; k < C::K_STEPS_PV / 2; ++k) {
+      const int kk = half * (C::K_STEPS_PV / 2) + k;
       mma_f16_ts(d_tmem, p_tmem + kk * 8, va + ((kk * 16 * C::SW_V) >> 4), C::IDESC_PV,
                  (accumulate || kk > 0) ? 1u : 0u);
+    }
+  };
+  // P_i arrives in two halves, each on its own barrier (one phase per step).
+  auto wait_p_and_issue = [&](int i, int stage, bool accumulate, int& p_cnt) -> bool {
+    const uint32_t parity = (p_cnt++) & 1;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      if (!wait_bounded(b.p_full(i, half), parity, abort_flag, limit)) return false;
+      FA_TRACE_EV(2, 30 + 2 * i + half, p_cnt - 1);
+      tc_fence_after();
+      issue_pv_half(i, stage, half, accumulate);
+    }
+    return true;
   };
 
   bool ok = true;
@@ -290,69 +331,251 @@ __device__ __noinline__ void mma_role(const FwdArgs& a, const Barriers& b, uint3
     const int q0 = t.tp * 256;
     const int n0 = kv_tiles(a, q0), n1 = kv_tiles(a, q0 + 128);
     const int nkv = n0 > n1 ? n0 : n1;
-    if (n0 > 0 && !wait_bounded(&b.q_full[0], (q_use0++) & 1, abort_flag, limit)) { ok = false; break; }
-    if (n1 > 0 && !wait_bounded(&b.q_full[1], (q_use1++) & 1, abort_flag, limit)) { ok = false; break; }
+    if (n0 > 0 && !wait_bounded(b.q_full(0), (q_use0++) & 1, abort_flag, limit)) { ok = false; break; }
+    if (n1 > 0 && !wait_bounded(b.q_full(1), (q_use1++) & 1, abort_flag, limit)) { ok = false; break; }
     int sk = kv_it % C::NS;
-    if (!wait_bounded(&b.kv_full[sk], (kv_it / C::NS) & 1, abort_flag, limit)) { ok = false; break; }
+    if (!wait_bounded(b.kv_full(sk), (kv_it / C::NS) & 1, abort_flag, limit)) { ok = false; break; }
     ++kv_it;
     tc_fence_after();
     if (n0 > 0) {
       issue_s(0, sk);
-      tc_commit(&b.s_full[0]);
-      if (n0 == 1) tc_commit(&b.q_empty[0]);
+      tc_commit(b.s_full(0));
+      if (n0 == 1) tc_commit(b.q_empty(0));
     }
     if (n1 > 0) {
       issue_s(1, sk);
-      tc_commit(&b.s_full[1]);
-      if (n1 == 1) tc_commit(&b.q_empty[1]);
+      tc_commit(b.s_full(1));
+      if (n1 == 1) tc_commit(b.q_empty(1));
     }
-    tc_commit(&b.kv_empty[sk]);
+    tc_commit(b.kv_empty(sk));
     for (int j = 0; j < nkv; ++j) {
       const int sv = kv_it % C::NS;
-      if (!wait_bounded(&b.kv_full[sv], (kv_it / C::NS) & 1, abort_flag, limit)) { ok = false; break; }
+      FA_TRACE_EV(2, 40, j);
+      if (!wait_bounded(b.kv_full(sv), (kv_it / C::NS) & 1, abort_flag, limit)) { ok = false; break; }
+      FA_TRACE_EV(2, 41, j);
       ++kv_it;
       tc_fence_after();
       if (j < n0) {
-        if (!wait_bounded(&b.p_full[0], (p_cnt0++) & 1, abort_flag, limit)) { ok = false; break; }
-        tc_fence_after();
-        issue_pv(0, sv, j > 0);
-        if (j == n0 - 1) tc_commit(&b.o_full[0]);
+        if (!wait_p_and_issue(0, sv, j > 0, p_cnt0)) { ok = false; break; }
+        if (j == n0 - 1) tc_commit(b.o_full(0));
       }
       const bool next = j + 1 < nkv;
       int sk2 = 0;
       if (next) {
         sk2 = kv_it % C::NS;
-        if (!wait_bounded(&b.kv_full[sk2], (kv_it / C::NS) & 1, abort_flag, limit)) { ok = false; break; }
+        FA_TRACE_EV(2, 42, j + 1);
+        if (!wait_bounded(b.kv_full(sk2), (kv_it / C::NS) & 1, abort_flag, limit)) { ok = false; break; }
+        FA_TRACE_EV(2, 43, j + 1);
         ++kv_it;
         tc_fence_after();
         if (j + 1 < n0) {
           issue_s(0, sk2);
-          tc_commit(&b.s_full[0]);
-          if (j + 1 == n0 - 1) tc_commit(&b.q_empty[0]);
+          tc_commit(b.s_full(0));
+          if (j + 1 == n0 - 1) tc_commit(b.q_empty(0));
         }
       }
       if (j < n1) {
-        if (!wait_bounded(&b.p_full[1], (p_cnt1++) & 1, abort_flag, limit)) { ok = false; break; }
-        tc_fence_after();
-        issue_pv(1, sv, j > 0);
-        if (j == n1 - 1) tc_commit(&b.o_full[1]);
+        if (!wait_p_and_issue(1, sv, j > 0, p_cnt1)) { ok = false; break; }
+        if (j == n1 - 1) tc_commit(b.o_full(1));
       }
-      tc_commit(&b.kv_empty[sv]);
+      tc_commit(b.kv_empty(sv));
       if (next) {
         if (j + 1 < n1) {
           issue_s(1, sk2);
-          tc_commit(&b.s_full[1]);
-          if (j + 1 == n1 - 1) tc_commit(&b.q_empty[1]);
+          tc_commit(b.s_full(1));
+          if (j + 1 == n1 - 1) tc_commit(b.q_empty(1));
         }
-        tc_commit(&b.kv_empty[sk2]);
+        tc_commit(b.kv_empty(sk2));
       }
     }
   }
   if (!ok) record_failure(a, abort_flag, kStatusMma);
   // Drain: all issued MMAs complete before tensor memory is released.
-  tc_commit(b.mma_done);
+  tc_commit(b.mma_done());
   volatile int never = 0;
-  if (!wait_bounded(b.mma_done, 0, &never, limit)) atomicOr(a.status, kStatusDrain);
+  if (!wait_bounded(b.mma_done(), 0, &never, limit)) atomicOr(a.status, kStatusDrain);
+}
+
+// ---------------------------------------------------------------- softmax
+// One warpgroup per Q tile; thread = query row.  Per K/V step: load the S
+// row from tensor memory, mask (last tile only), row max, deferred rescale
+// of O, p = 2^(s * scale * log2 e - m), row sum, P (16-bit) back into the S
+// columns in two halves.  Epilogue: O / l to global memory, LSE.
+template <int D, int ELEM>
+__device__ __forceinline__ void softmax_role(const FwdArgs& a, const Bars<FwdCfg<D, ELEM>::NS> b, uint32_t tmem,
+                                             int warp, int lane, volatile int* abort_flag) {
+  using C = FwdCfg<D, ELEM>;
+  const uint64_t limit = a.wait_limit_ns;
+  const int wg = warp >> 2;            // which Q tile
+  const int wq = warp & 3;             // warp within the warpgroup -> TMEM lanes
+  const int row = wq * 32 + lane;      // query row within the Q tile
+  const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+  const uint32_t t_s = tmem + lane_off + (wg ? C::S_COL1 : C::S_COL0);
+  const uint32_t t_o = tmem + lane_off + (wg ? C::O_COL1 : C::O_COL0);
+  const uint32_t s_full = b.s_full(wg);
+  const uint32_t o_full = b.o_full(wg);
+  int s_cnt = 0, o_cnt = 0;
+  FA_TRACE_DECL;
+  using OutT = typename std::conditional<ELEM == kElemF16, __half, __nv_bfloat16>::type;
+
+  auto wait_warp = [&](uint32_t bar, int parity) -> bool {
+    bool ok = wait_bounded(bar, parity & 1, abort_flag, limit);
+    return __all_sync(0xffffffffu, ok);
+  };
+
+  auto run = [&]() -> bool {
+    for (int w = blockIdx.x; w < a.n_work; w += gridDim.x) {
+      const WorkTile t = decode_work(a, w);
+      const int q_start = t.tp * 256 + wg * 128;
+      const int nkv = kv_tiles(a, q_start);
+      if (nkv == 0) continue;
+      const int qrow = q_start + row;
+      float sl2_q = a.scale_log2;
+      if constexpr (ELEM == kElemE4M3) sl2_q = a.scale_log2 / a.q_scale[t.bh * a.n_qtiles + (q_start >> 7)];
+      float m = -INFINITY;  // running max, log2 units of the scaled score
+      float l = 0.f;        // running sum of exponentials
+      for (int j = 0; j < nkv; ++j) {
+        if (lane == 0 && wq == 0) FA_TRACE_EV(wg, 0 + 10 * wg, j);
+        if (!wait_warp(s_full, s_cnt)) return false;
+        ++s_cnt;
+        tc_fence_after();
+        if (lane == 0 && wq == 0) FA_TRACE_EV(wg, 1 + 10 * wg, j);
+        float sl2 = sl2_q;
+        if constexpr (ELEM == kElemE4M3) sl2 = sl2_q / a.k_scale[t.bh * a.n_qtiles + j];
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, sr[c]);
+        tmem_ld_wait(sr[0]);
+        reg_tie(sr[1]);
+        reg_tie(sr[2]);
+        reg_tie(sr[3]);
+#define FA_S(c) __uint_as_float(sr[(c) >> 5][(c) & 31])
+        if (j == nkv - 1) {
+          // last tile of this row block: keys past the sequence end, and
+          // (causal) keys after the query, become -inf
+          int limit_key = a.N - 1;
+          if (a.causal && qrow < limit_key) limit_key = qrow;
+          const int kbase = j * 128;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (kbase + c > limit_key) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+        }
+        float mx0 = FA_S(0), mx1 = FA_S(1), mx2 = FA_S(2), mx3 = FA_S(3);
+#pragma unroll
+        for (int c = 4; c < 124; c += 8) {
+          mx0 = fmax3(mx0, FA_S(c), FA_S(c + 1));
+          mx1 = fmax3(mx1, FA_S(c + 2), FA_S(c + 3));
+          mx2 = fmax3(mx2, FA_S(c + 4), FA_S(c + 5));
+          mx3 = fmax3(mx3, FA_S(c + 6), FA_S(c + 7));
+        }
+        mx0 = fmax3(mx0, FA_S(124), FA_S(125));
+        mx1 = fmax3(mx1, FA_S(126), FA_S(127));
+        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+        if (lane == 0 && wq == 0) FA_TRACE_EV(wg, 2 + 10 * wg, j);
+        if (j == 0) {
+          m = mx;
+        } else {
+          const bool need = mx - m > C::TAU;
+          if (__any_sync(0xffffffffu, need)) {
+            const float m_new = fmaxf(m, mx);
+            const float alpha = ex2_approx(m - m_new);
+            m = m_new;
+            l *= alpha;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t orr[32];
+              tmem_ld32(t_o + c * 32, orr);
+              tmem_ld_wait(orr);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+              tmem_st32(t_o + c * 32, orr);
+            }
+          }
+        }
+        // p = 2^(s * sl2 - m), two columns per packed instruction; the column
+        // pairs marked in POLY_MASK use the polynomial exp2, the rest the
+        // special-function unit.  P goes to tensor memory in two halves
+        // (keys 0-63, then 64-127); the MMA warp starts P V on the first half
+        // while the second is computed.
+        const uint64_t sl2x2 = pack2(sl2, sl2);
+        const uint64_t negm2 = pack2(-m, -m);
+        uint64_t acc_a = pack2(0.f, 0.f), acc_b = pack2(0.f, 0.f);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+#pragma unroll
+          for (int c = 2 * half; c < 2 * half + 2; ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const uint64_t x2 = ffma2(pack2(FA_S(c * 32 + 2 * e), FA_S(c * 32 + 2 * e + 1)), sl2x2, negm2);
+              uint64_t p2;
+              if ((C::POLY_MASK >> e) & 1u) {
+                p2 = exp2_poly2(x2);
+              } else {
+                float x0, x1;
+                unpack2(x2, x0, x1);
+                p2 = pack2(ex2_approx(x0), ex2_approx(x1));
+              }
+              if (e & 1)
+                acc_b = fadd2(acc_b, p2);
+              else
+                acc_a = fadd2(acc_a, p2);
+              float p0, p1;
+              unpack2(p2, p0, p1);
+              if constexpr (ELEM == kElemF16)
+                pk[e] = pack_f16x2(p0, p1);
+              else
+                pk[e] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(t_s + c * 16, pk);
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(b.p_full(wg, half));
+          if (lane == 0 && wq == 0) FA_TRACE_EV(wg, 3 + half + 10 * wg, j);
+        }
+#undef FA_S
+        {
+          float a0, a1, b0, b1;
+          unpack2(acc_a, a0, a1);
+          unpack2(acc_b, b0, b1);
+          l += (a0 + a1) + (b0 + b1);
+        }
+      }
+      // epilogue: O / l -> global, LSE
+      if (!wait_warp(o_full, o_cnt)) return false;
+      ++o_cnt;
+      if (lane == 0 && wq == 0) FA_TRACE_EV(wg, 5 + 10 * wg, 0);
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      OutT* orow = reinterpret_cast<OutT*>(a.o) + (static_cast<size_t>(t.bh) * a.N + qrow) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t orr[32];
+        tmem_ld32(t_o + c * 32, orr);
+        tmem_ld_wait(orr);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float v0 = __uint_as_float(orr[2 * e]) * inv_l;
+          const float v1 = __uint_as_float(orr[2 * e + 1]) * inv_l;
+          pk[e] = (ELEM == kElemF16) ? pack_f16x2(v0, v1) : pack_bf16x2(v0, v1);
+        }
+        if (qrow < a.N) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      }
+      if (lane == 0 && wq == 0) FA_TRACE_EV(wg, 6 + 10 * wg, 0);
+      if (a.lse != nullptr && qrow < a.N)
+        a.lse[static_cast<size_t>(t.bh) * a.N + qrow] = (m + __log2f(l)) * 0.69314718055994531f;
+    }
+    return true;
+  };
+  if (!run()) record_failure(a, abort_flag, kStatusSoftmax);
+  tc_fence_before();
 }
 
 template <int D, int ELEM>
@@ -366,19 +589,9 @@ __global__ void __launch_bounds__(384, 1)
   volatile int* abort_flag = &abort_flag_storage;
 
   const uint32_t raw_addr = smem_u32(smem_raw);
-  uint8_t* base = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
-  uint8_t* sQ = base;                       // [2][Q_TILE]
-  uint8_t* sKV = base + 2 * C::Q_TILE;      // [NS][STAGE]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + C::TILE_BYTES);
-  Barriers b;
-  b.q_full = bars;
-  b.q_empty = bars + 2;
-  b.kv_full = bars + 4;
-  b.kv_empty = bars + 4 + C::NS;
-  b.s_full = bars + 4 + 2 * C::NS;
-  b.p_full = b.s_full + 2;
-  b.o_full = b.p_full + 2;
-  b.mma_done = b.o_full + 2;
+  const uint32_t sQ = (raw_addr + 1023u) & ~1023u;   // [2][Q_TILE], 1024-byte aligned for the swizzle
+  const uint32_t sKV = sQ + 2 * C::Q_TILE;           // [NS][STAGE]
+  const Bars<C::NS> b{sQ + C::TILE_BYTES};
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -386,17 +599,18 @@ __global__ void __launch_bounds__(384, 1)
   if (threadIdx.x == 0) {
     abort_flag_storage = 0;
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&b.q_full[i], 1);
-      mbar_init(&b.q_empty[i], 1);
-      mbar_init(&b.s_full[i], 1);
-      mbar_init(&b.p_full[i], 4);
-      mbar_init(&b.o_full[i], 1);
+      mbar_init(b.q_full(i), 1);
+      mbar_init(b.q_empty(i), 1);
+      mbar_init(b.s_full(i), 1);
+      mbar_init(b.p_full(i, 0), 4);
+      mbar_init(b.p_full(i, 1), 4);
+      mbar_init(b.o_full(i), 1);
     }
     for (int s = 0; s < C::NS; ++s) {
-      mbar_init(&b.kv_full[s], 1);
-      mbar_init(&b.kv_empty[s], 1);
+      mbar_init(b.kv_full(s), 1);
+      mbar_init(b.kv_empty(s), 1);
     }
-    mbar_init(b.mma_done, 1);
+    mbar_init(b.mma_done(), 1);
     fence_barrier_init();
   }
   if (warp == C::MMA_WARP) {
@@ -407,7 +621,6 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_holder;
-  const uint64_t limit = a.wait_limit_ns;
 
   // Each role's code sits inside the branch that set its register budget, so
   // the compiler allocates the softmax code for REG_SOFTMAX registers.
@@ -416,148 +629,11 @@ __global__ void __launch_bounds__(384, 1)
     if (warp == C::LOAD_WARP && lane == 0)
       producer_role<D, ELEM>(a, b, sQ, sKV, &map_q, &map_k, &map_v, abort_flag);
     else if (warp == C::MMA_WARP && lane == 0)
-      mma_role<D, ELEM>(a, b, smem_u32(sQ), smem_u32(sKV), tmem, abort_flag);
+      mma_role<D, ELEM>(a, b, sQ, sKV, tmem, abort_flag);
     // warps 10 and 11 only give their registers away
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(C::REG_SOFTMAX));
-    // ------------------------------------------------------------ softmax
-    const int wg = warp >> 2;            // which Q tile
-    const int wq = warp & 3;             // warp within the warpgroup -> TMEM lanes
-    const int row = wq * 32 + lane;      // query row within the Q tile
-    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t t_s = tmem + lane_off + (wg ? C::S_COL1 : C::S_COL0);
-    const uint32_t t_o = tmem + lane_off + (wg ? C::O_COL1 : C::O_COL0);
-    uint64_t* s_full = &b.s_full[wg];
-    uint64_t* p_full = &b.p_full[wg];
-    uint64_t* o_full = &b.o_full[wg];
-    int s_cnt = 0, o_cnt = 0;
-    using OutT = typename std::conditional<ELEM == kElemF16, __half, __nv_bfloat16>::type;
-
-    auto wait_warp = [&](uint64_t* bar, int parity) -> bool {
-      bool ok = wait_bounded(bar, parity & 1, abort_flag, limit);
-      return __all_sync(0xffffffffu, ok);
-    };
-
-    auto run = [&]() -> bool {
-      for (int w = blockIdx.x; w < a.n_work; w += gridDim.x) {
-        const WorkTile t = decode_work(a, w);
-        const int q_start = t.tp * 256 + wg * 128;
-        const int nkv = kv_tiles(a, q_start);
-        if (nkv == 0) continue;
-        const int qrow = q_start + row;
-        float sl2_q = a.scale_log2;
-        if constexpr (ELEM == kElemE4M3) sl2_q = a.scale_log2 / a.q_scale[t.bh * a.n_qtiles + (q_start >> 7)];
-        float m = -INFINITY;  // running max, log2 units of the scaled score
-        float l = 0.f;        // running sum of exponentials
-        for (int j = 0; j < nkv; ++j) {
-          if (!wait_warp(s_full, s_cnt)) return false;
-          ++s_cnt;
-          tc_fence_after();
-          float sl2 = sl2_q;
-          if constexpr (ELEM == kElemE4M3) sl2 = sl2_q / a.k_scale[t.bh * a.n_qtiles + j];
-          uint32_t sr[4][32];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, sr[c]);
-          tmem_ld_wait(sr[0]);
-          reg_tie(sr[1]);
-          reg_tie(sr[2]);
-          reg_tie(sr[3]);
-#define FA_S(c) __uint_as_float(sr[(c) >> 5][(c) & 31])
-          if (j == nkv - 1) {
-            // last tile of this row block: keys past the sequence end, and
-            // (causal) keys after the query, become -inf
-            int limit_key = a.N - 1;
-            if (a.causal && qrow < limit_key) limit_key = qrow;
-            const int kbase = j * 128;
-#pragma unroll
-            for (int c = 0; c < 128; ++c)
-              if (kbase + c > limit_key) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
-          }
-          float mx0 = FA_S(0), mx1 = FA_S(1), mx2 = FA_S(2), mx3 = FA_S(3);
-#pragma unroll
-          for (int c = 4; c < 128; c += 4) {
-            mx0 = fmaxf(mx0, FA_S(c));
-            mx1 = fmaxf(mx1, FA_S(c + 1));
-            mx2 = fmaxf(mx2, FA_S(c + 2));
-            mx3 = fmaxf(mx3, FA_S(c + 3));
-          }
-          const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
-          if (j == 0) {
-            m = mx;
-          } else {
-            const bool need = mx - m > C::TAU;
-            if (__any_sync(0xffffffffu, need)) {
-              const float m_new = fmaxf(m, mx);
-              const float alpha = ex2_approx(m - m_new);
-              m = m_new;
-              l *= alpha;
-#pragma unroll
-              for (int c = 0; c < D / 32; ++c) {
-                uint32_t orr[32];
-                tmem_ld32(t_o + c * 32, orr);
-                tmem_ld_wait(orr);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-                tmem_st32(t_o + c * 32, orr);
-              }
-            }
-          }
-          const float neg_m = -m;
-          float sum0 = 0.f, sum1 = 0.f;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float p0 = ex2_approx(fmaf(FA_S(c * 32 + 2 * e), sl2, neg_m));
-              const float p1 = ex2_approx(fmaf(FA_S(c * 32 + 2 * e + 1), sl2, neg_m));
-              sum0 += p0;
-              sum1 += p1;
-              if constexpr (ELEM == kElemF16)
-                pk[e] = pack_f16x2(p0, p1);
-              else
-                pk[e] = pack_bf16x2(p0, p1);
-            }
-            tmem_st16(t_s + c * 16, pk);
-          }
-#undef FA_S
-          l += sum0 + sum1;
-          tmem_st_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(p_full);
-        }
-        // epilogue: O / l -> global, LSE
-        if (!wait_warp(o_full, o_cnt)) return false;
-        ++o_cnt;
-        tc_fence_after();
-        const float inv_l = 1.f / l;
-        OutT* orow = reinterpret_cast<OutT*>(a.o) + (static_cast<size_t>(t.bh) * a.N + qrow) * D;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t orr[32];
-          tmem_ld32(t_o + c * 32, orr);
-          tmem_ld_wait(orr);
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float v0 = __uint_as_float(orr[2 * e]) * inv_l;
-            const float v1 = __uint_as_float(orr[2 * e + 1]) * inv_l;
-            pk[e] = (ELEM == kElemF16) ? pack_f16x2(v0, v1) : pack_bf16x2(v0, v1);
-          }
-          if (qrow < a.N) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-          }
-        }
-        if (a.lse != nullptr && qrow < a.N)
-          a.lse[static_cast<size_t>(t.bh) * a.N + qrow] = (m + __log2f(l)) * 0.69314718055994531f;
-      }
-      return true;
-    };
-    if (!run()) record_failure(a, abort_flag, kStatusSoftmax);
-    tc_fence_before();
+    softmax_role<D, ELEM>(a, b, tmem, warp, lane, abort_flag);
   }
 
   __syncthreads();

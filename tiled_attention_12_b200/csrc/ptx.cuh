@@ -22,31 +22,31 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 }
 
 // ---------------------------------------------------------------- mbarrier
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+// Barriers are addressed by their 32-bit shared-memory address.
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}\n"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
 }
@@ -54,7 +54,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Waits for the phase with the given parity to complete.  Returns false when
 // `abort_flag` becomes nonzero or `limit_ns` elapses; the caller then records
 // the failure and leaves its loop.  Never spins without bound.
-__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                              uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
@@ -69,12 +69,12 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, vol
 // 3-D tiled bulk tensor load global -> shared, completion counted in bytes on
 // `bar`.  Coordinates are innermost first; c0 * element size is a multiple of
 // 16 bytes at every call site (tile starts are multiples of the box width).
-__device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int c0,
-                                            int c1, int c2) {
+__device__ __forceinline__ void tma_load_3d(uint32_t smem_dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
+                                            int c2) {
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
 
@@ -102,10 +102,8 @@ __device__ __forceinline__ void tc_fence_after() {
 }
 // Arrive on `bar` once every tcgen05 operation this thread issued so far has
 // completed.
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
 
 #define FA_R8(a, i) "=r"(a[i]), "=r"(a[i + 1]), "=r"(a[i + 2]), "=r"(a[i + 3]), \
@@ -230,3 +228,96 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 }
 
 }  // namespace fa
+
+namespace fa {
+
+// ---------------------------------------------------------------- packed fp32
+// Two fp32 values in one 64-bit register pair; the f32x2 forms below issue
+// one instruction for both lanes.
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for two lanes without the special-function unit.
+//
+// Range reduction (the standard Cody-Waite split, trivial for base 2):
+// x = n + f with n = round-to-nearest(x), obtained exactly by adding and
+// subtracting 1.5 * 2^23, and f = x - n in [-1/2, 1/2].  2^f comes from a
+// degree-3 polynomial whose coefficients are the relative-error minimax fit
+// on [-1/2, 1/2] found by a Remez exchange (max relative error 7.5e-5, well
+// under the 2^-9 of the bf16 P it feeds).  2^n is applied by adding n to the
+// exponent field: the integer bits of (x + 1.5 * 2^23) shifted left by 23
+// are exactly n << 23.  Inputs below -126 are clamped so the exponent field
+// cannot underflow into the sign bit; they return a value below 2^-125.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  float x0, x1;
+  unpack2(x2, x0, x1);
+  const uint64_t xc = pack2(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const uint64_t r = fadd2(xc, pack2(12582912.0f, 12582912.0f));
+  const uint64_t n = fadd2(r, pack2(-12582912.0f, -12582912.0f));
+  const uint64_t f = ffma2(n, pack2(-1.0f, -1.0f), xc);
+  uint64_t p = ffma2(pack2(0.0551716685295105f, 0.0551716685295105f), f,
+                     pack2(0.2426111251115799f, 0.2426111251115799f));
+  p = ffma2(p, f, pack2(0.6932609677314758f, 0.6932609677314758f));
+  p = ffma2(p, f, pack2(0.9999280571937561f, 0.9999280571937561f));
+  float p0, p1, r0, r1;
+  unpack2(p, p0, p1);
+  unpack2(r, r0, r1);
+  return pack2(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(r0) << 23)),
+               __uint_as_float(__float_as_uint(p1) + (__float_as_uint(r1) << 23)));
+}
+
+}  // namespace fa
+
+// ---------------------------------------------------------------- tracing
+// Compile with -DFA_TRACE to record (event, step, SM clock) triples from CTA 0
+// into a device array; the trace-enabled build exports fa_trace_read() to
+// copy it out.  Each tracing thread owns a slice of the array (`slot` 0..7)
+// and writes it with plain stores, so tracing adds no atomics or waits to
+// the traced path.  Without FA_TRACE the macro expands to nothing.
+#ifdef FA_TRACE
+#ifndef FA_TRACE_CAP
+#define FA_TRACE_CAP 16384
+#endif
+namespace fa {
+// one copy per translation unit; the reader sits in the same unit as the
+// kernels it traces
+static __device__ unsigned long long g_fa_trace[FA_TRACE_CAP];
+}  // namespace fa
+#define FA_TRACE_DECL unsigned trace_i_ = 0
+#define FA_TRACE_EV(slot, id, step)                                                                      \
+  do {                                                                                                   \
+    if (blockIdx.x == 0 && trace_i_ < FA_TRACE_CAP / 8)                                                  \
+      ::fa::g_fa_trace[(slot) * (FA_TRACE_CAP / 8) + trace_i_++] =                                       \
+          (static_cast<unsigned long long>(id) << 56) |                                                  \
+          (static_cast<unsigned long long>((step) & 0xFFFF) << 40) |                                     \
+          (static_cast<unsigned long long>(clock64()) & 0xFFFFFFFFFFull);                                \
+  } while (0)
+#else
+#define FA_TRACE_DECL \
+  do {                \
+  } while (0)
+#define FA_TRACE_EV(slot, id, step) \
+  do {                              \
+  } while (0)
+#endif
