@@ -42,6 +42,10 @@
 #ifndef FA_POLY_MASK
 #define FA_POLY_MASK 0x4924u
 #endif
+// 1: the softmax hands P to the MMA warp in two halves (keys 0-63, 64-127)
+#ifndef FA_SPLIT_P
+#define FA_SPLIT_P 1
+#endif
 // shared-memory bytes for the Q tiles plus the K/V ring (sets the ring depth)
 #ifndef FA_SMEM_FOR_TILES
 #define FA_SMEM_FOR_TILES (200 * 1024)
@@ -91,7 +95,7 @@ struct FwdCfg {
   static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;  // K/V ring depth
   static_assert(NS >= 2, "ring too shallow");
   static constexpr int TILE_BYTES = 2 * Q_TILE + NS * STAGE;
-  static constexpr int NUM_BARS = 13 + 2 * NS;
+  static constexpr int NUM_BARS = 17 + 2 * NS;
   // at least 120 KB so that two CTAs never share an SM (each holds all 512
   // tensor-memory columns; a second resident CTA would only wait)
   static constexpr int SMEM_NEED = 1024 + TILE_BYTES + 8 * NUM_BARS;
@@ -100,8 +104,16 @@ struct FwdCfg {
   static constexpr int K_STEPS_QK = QK_ROW / 32;   // 32 bytes of K per S MMA (16 x 16-bit or 32 x 8-bit)
   static constexpr int K_STEPS_PV = BN / 16;       // 16 keys per P V MMA
   static constexpr int THREADS = 384;  // 3 warpgroups
-  static constexpr int MMA_WARP = 8;
-  static constexpr int LOAD_WARP = 9;  // warps 10, 11 only rebalance registers
+  static constexpr int MMA_WARP = 8;    // MMA issuer (Q tile 0 when decoupled); allocates tensor memory
+  static constexpr int LOAD_WARP = 9;
+  static constexpr int MMA_WARP1 = 10;  // Q tile 1's MMA issuer when decoupled; warp 11 only rebalances
+  // Decoupled layout (d <= 64): P has tensor-memory columns of its own, so
+  // S_i(j+1) can be computed while the softmax still works on step j, and each
+  // Q tile gets its own MMA issuer.  At d = 128 the 512 columns only hold S and
+  // O for both tiles, so P overwrites S and one issuer keeps the two tiles in
+  // ping-pong order.
+  static constexpr bool DECOUPLED = D <= 64;
+  static constexpr int ISSUERS = DECOUPLED ? 2 : 1;
   // Register split (setmaxnreg): the block launches with LAUNCH_REGS per
   // thread; the two softmax warpgroups then take REG_SOFTMAX and the
   // MMA/TMA warpgroup gives back down to REG_OTHER.  The shares must add up
@@ -111,7 +123,9 @@ struct FwdCfg {
   static constexpr int REG_OTHER = 88;
   static_assert(2 * 128 * REG_SOFTMAX + 128 * REG_OTHER == THREADS * LAUNCH_REGS, "register split");
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t S_COL0 = 0, S_COL1 = 128, O_COL0 = 256, O_COL1 = 256 + D;
+  static constexpr uint32_t S_COL0 = 0, S_COL1 = 128;
+  static constexpr uint32_t P_COL0 = DECOUPLED ? 256 : S_COL0, P_COL1 = DECOUPLED ? 320 : S_COL1;
+  static constexpr uint32_t O_COL0 = DECOUPLED ? 384 : 256, O_COL1 = O_COL0 + D;
   static_assert(O_COL1 + D <= TMEM_COLS, "tensor memory budget exceeded");
   static constexpr uint32_t IDESC_QK =
       instr_desc(ELEM == kElemBF16 ? 1u : 0u, ELEM == kElemBF16 ? 1u : 0u, 0u, BM, BN);
@@ -144,7 +158,11 @@ struct Bars {
   }
   __device__ __forceinline__ uint32_t o_full(int i) const { return base + 8u * (10 + 2 * NS + i); }  // MMA -> epilogue
   __device__ __forceinline__ uint32_t mma_done() const { return base + 8u * (12 + 2 * NS); }
-  static constexpr int COUNT = 13 + 2 * NS;
+  // decoupled layout only: softmax i has read S_i (4 warp arrivals) / the
+  // MMA that read P_i and updated O_i has completed
+  __device__ __forceinline__ uint32_t s_free(int i) const { return base + 8u * (13 + 2 * NS + i); }
+  __device__ __forceinline__ uint32_t p_free(int i) const { return base + 8u * (15 + 2 * NS + i); }
+  static constexpr int COUNT = 17 + 2 * NS;
 };
 
 struct WorkTile {
@@ -312,14 +330,17 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const Bars<FwdCfg<D, 
                  (accumulate || kk > 0) ? 1u : 0u);
     }
   };
-  // P_i arrives in two halves, each on its own barrier (one phase per step).
+  // P_i arrives in two halves, each on its own barrier (one phase per step),
+  // or whole on the first barrier.
   auto wait_p_and_issue = [&](int i, int stage, bool accumulate, int& p_cnt) -> bool {
     const uint32_t parity = (p_cnt++) & 1;
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
-      if (!wait_bounded(b.p_full(i, half), parity, abort_flag, limit)) return false;
-      FA_TRACE_EV(2, 30 + 2 * i + half, p_cnt - 1);
-      tc_fence_after();
+      if (FA_SPLIT_P || half == 0) {
+        if (!wait_bounded(b.p_full(i, half), parity, abort_flag, limit)) return false;
+        FA_TRACE_EV(2, 30 + 2 * i + half, p_cnt - 1);
+        tc_fence_after();
+      }
       issue_pv_half(i, stage, half, accumulate);
     }
     return true;
@@ -399,8 +420,164 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const Bars<FwdCfg<D, 
 // ---------------------------------------------------------------- softmax
 // One warpgroup per Q tile; thread = query row.  Per K/V step: load the S
 // row from tensor memory, mask (last tile only), row max, deferred rescale
-// of O, p = 2^(s * scale * log2 e - m), row sum, P (16-bit) back into the S
-// columns in two halves.  Epilogue: O / l to global memory, LSE.
+// of O, p = 2^(s * scale * log2 e - m), row sum, 16-bit P into tensor memory.
+// Epilogue: O / l to global memory, LSE.
+
+// The S row of this thread: 128 fp32 scores in four 32-column loads.
+__device__ __forceinline__ void load_s_row(uint32_t t_s, uint32_t (&sr)[4][32]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, sr[c]);
+  tmem_ld_wait(sr[0]);
+  reg_tie(sr[1]);
+  reg_tie(sr[2]);
+  reg_tie(sr[3]);
+}
+
+#define FA_S(c) __uint_as_float(sr[(c) >> 5][(c) & 31])
+
+// Keys past limit_key (the sequence end, or the query itself when causal)
+// become -inf.  Only the last K/V tile of a row block can hold such keys.
+__device__ __forceinline__ void mask_row(uint32_t (&sr)[4][32], int kbase, int limit_key) {
+#pragma unroll
+  for (int c = 0; c < 128; ++c)
+    if (kbase + c > limit_key) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+}
+
+__device__ __forceinline__ float row_max(const uint32_t (&sr)[4][32]) {
+  float mx0 = FA_S(0), mx1 = FA_S(1), mx2 = FA_S(2), mx3 = FA_S(3);
+#pragma unroll
+  for (int c = 4; c < 124; c += 8) {
+    mx0 = fmax3(mx0, FA_S(c), FA_S(c + 1));
+    mx1 = fmax3(mx1, FA_S(c + 2), FA_S(c + 3));
+    mx2 = fmax3(mx2, FA_S(c + 4), FA_S(c + 5));
+    mx3 = fmax3(mx3, FA_S(c + 6), FA_S(c + 7));
+  }
+  mx0 = fmax3(mx0, FA_S(124), FA_S(125));
+  mx1 = fmax3(mx1, FA_S(126), FA_S(127));
+  return fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+}
+
+// O row *= alpha in tensor memory (the deferred correction step).
+template <int D>
+__device__ __forceinline__ void rescale_o(uint32_t t_o, float alpha) {
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t orr[32];
+    tmem_ld32(t_o + c * 32, orr);
+    tmem_ld_wait(orr);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+    tmem_st32(t_o + c * 32, orr);
+  }
+}
+
+// p = 2^(s * sl2 - m) for the 64 columns of `half`, two per packed
+// instruction; column pairs marked in POLY_MASK use the FMA-pipe polynomial,
+// the rest the special-function unit.  The 16-bit P goes to tensor memory at
+// t_p (16 columns per 32 scores) and the fp32 sums into acc_a / acc_b.
+template <int ELEM, uint32_t POLY_MASK>
+__device__ __forceinline__ void exp_store_half(const uint32_t (&sr)[4][32], int half, uint64_t sl2x2,
+                                               uint64_t negm2, uint32_t t_p, uint64_t& acc_a, uint64_t& acc_b) {
+#pragma unroll
+  for (int c = 2 * half; c < 2 * half + 2; ++c) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const uint64_t x2 = ffma2(pack2(FA_S(c * 32 + 2 * e), FA_S(c * 32 + 2 * e + 1)), sl2x2, negm2);
+      uint64_t p2;
+      if ((POLY_MASK >> e) & 1u) {
+        p2 = exp2_poly2(x2);
+      } else {
+        float x0, x1;
+        unpack2(x2, x0, x1);
+        p2 = pack2(ex2_approx(x0), ex2_approx(x1));
+      }
+      if (e & 1)
+        acc_b = fadd2(acc_b, p2);
+      else
+        acc_a = fadd2(acc_a, p2);
+      float p0, p1;
+      unpack2(p2, p0, p1);
+      if constexpr (ELEM == kElemF16)
+        pk[e] = pack_f16x2(p0, p1);
+      else
+        pk[e] = pack_bf16x2(p0, p1);
+    }
+    tmem_st16(t_p + c * 16, pk);
+  }
+}
+
+// Same as exp_store_half for all 128 columns, but the packed P stays in
+// registers (pk[chunk][16]) so it can be stored later.
+template <int ELEM, uint32_t POLY_MASK>
+__device__ __forceinline__ void exp_to_regs(const uint32_t (&sr)[4][32], uint64_t sl2x2, uint64_t negm2,
+                                            uint32_t (&pk)[4][16], uint64_t& acc_a, uint64_t& acc_b) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const uint64_t x2 = ffma2(pack2(FA_S(c * 32 + 2 * e), FA_S(c * 32 + 2 * e + 1)), sl2x2, negm2);
+      uint64_t p2;
+      if ((POLY_MASK >> e) & 1u) {
+        p2 = exp2_poly2(x2);
+      } else {
+        float x0, x1;
+        unpack2(x2, x0, x1);
+        p2 = pack2(ex2_approx(x0), ex2_approx(x1));
+      }
+      if (e & 1)
+        acc_b = fadd2(acc_b, p2);
+      else
+        acc_a = fadd2(acc_a, p2);
+      float p0, p1;
+      unpack2(p2, p0, p1);
+      if constexpr (ELEM == kElemF16)
+        pk[c][e] = pack_f16x2(p0, p1);
+      else
+        pk[c][e] = pack_bf16x2(p0, p1);
+    }
+  }
+}
+
+#undef FA_S
+
+__device__ __forceinline__ float sum_acc(uint64_t acc_a, uint64_t acc_b) {
+  float a0, a1, b0, b1;
+  unpack2(acc_a, a0, a1);
+  unpack2(acc_b, b0, b1);
+  return (a0 + a1) + (b0 + b1);
+}
+
+// O / l of this thread's row to global memory (16-byte stores), and LSE.
+template <int D, int ELEM>
+__device__ __forceinline__ void epilogue_row(const FwdArgs& a, uint32_t t_o, int bh, int qrow, float m, float l) {
+  using OutT = typename std::conditional<ELEM == kElemF16, __half, __nv_bfloat16>::type;
+  const float inv_l = 1.f / l;
+  OutT* orow = reinterpret_cast<OutT*>(a.o) + (static_cast<size_t>(bh) * a.N + qrow) * D;
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t orr[32];
+    tmem_ld32(t_o + c * 32, orr);
+    tmem_ld_wait(orr);
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float v0 = __uint_as_float(orr[2 * e]) * inv_l;
+      const float v1 = __uint_as_float(orr[2 * e + 1]) * inv_l;
+      pk[e] = (ELEM == kElemF16) ? pack_f16x2(v0, v1) : pack_bf16x2(v0, v1);
+    }
+    if (qrow < a.N) {
+      uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+    }
+  }
+  if (a.lse != nullptr && qrow < a.N)
+    a.lse[static_cast<size_t>(bh) * a.N + qrow] = (m + __log2f(l)) * 0.69314718055994531f;
+}
+
+// Aliased layout (d = 128): P overwrites the first 64 columns of S, and the
+// MMA warp's order (S_i(j+1) after P_i(j) V) sequences the reuse.
 template <int D, int ELEM>
 __device__ __forceinline__ void softmax_role(const FwdArgs& a, const Bars<FwdCfg<D, ELEM>::NS> b, uint32_t tmem,
                                              int warp, int lane, volatile int* abort_flag) {
@@ -416,7 +593,6 @@ __device__ __forceinline__ void softmax_role(const FwdArgs& a, const Bars<FwdCfg
   const uint32_t o_full = b.o_full(wg);
   int s_cnt = 0, o_cnt = 0;
   FA_TRACE_DECL;
-  using OutT = typename std::conditional<ELEM == kElemF16, __half, __nv_bfloat16>::type;
 
   auto wait_warp = [&](uint32_t bar, int parity) -> bool {
     bool ok = wait_bounded(bar, parity & 1, abort_flag, limit);
@@ -443,139 +619,245 @@ __device__ __forceinline__ void softmax_role(const FwdArgs& a, const Bars<FwdCfg
         float sl2 = sl2_q;
         if constexpr (ELEM == kElemE4M3) sl2 = sl2_q / a.k_scale[t.bh * a.n_qtiles + j];
         uint32_t sr[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, sr[c]);
-        tmem_ld_wait(sr[0]);
-        reg_tie(sr[1]);
-        reg_tie(sr[2]);
-        reg_tie(sr[3]);
-#define FA_S(c) __uint_as_float(sr[(c) >> 5][(c) & 31])
-        if (j == nkv - 1) {
-          // last tile of this row block: keys past the sequence end, and
-          // (causal) keys after the query, become -inf
-          int limit_key = a.N - 1;
-          if (a.causal && qrow < limit_key) limit_key = qrow;
-          const int kbase = j * 128;
-#pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (kbase + c > limit_key) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
-        }
-        float mx0 = FA_S(0), mx1 = FA_S(1), mx2 = FA_S(2), mx3 = FA_S(3);
-#pragma unroll
-        for (int c = 4; c < 124; c += 8) {
-          mx0 = fmax3(mx0, FA_S(c), FA_S(c + 1));
-          mx1 = fmax3(mx1, FA_S(c + 2), FA_S(c + 3));
-          mx2 = fmax3(mx2, FA_S(c + 4), FA_S(c + 5));
-          mx3 = fmax3(mx3, FA_S(c + 6), FA_S(c + 7));
-        }
-        mx0 = fmax3(mx0, FA_S(124), FA_S(125));
-        mx1 = fmax3(mx1, FA_S(126), FA_S(127));
-        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+        load_s_row(t_s, sr);
+        if (j == nkv - 1) mask_row(sr, j * 128, (a.causal && qrow < a.N - 1) ? qrow : a.N - 1);
+        const float mx = row_max(sr) * sl2;
         if (lane == 0 && wq == 0) FA_TRACE_EV(wg, 2 + 10 * wg, j);
         if (j == 0) {
           m = mx;
-        } else {
-          const bool need = mx - m > C::TAU;
-          if (__any_sync(0xffffffffu, need)) {
-            const float m_new = fmaxf(m, mx);
-            const float alpha = ex2_approx(m - m_new);
-            m = m_new;
-            l *= alpha;
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t orr[32];
-              tmem_ld32(t_o + c * 32, orr);
-              tmem_ld_wait(orr);
-#pragma unroll
-              for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-              tmem_st32(t_o + c * 32, orr);
-            }
-          }
+        } else if (__any_sync(0xffffffffu, mx - m > C::TAU)) {
+          const float m_new = fmaxf(m, mx);
+          const float alpha = ex2_approx(m - m_new);
+          m = m_new;
+          l *= alpha;
+          rescale_o<D>(t_o, alpha);
         }
-        // p = 2^(s * sl2 - m), two columns per packed instruction; the column
-        // pairs marked in POLY_MASK use the polynomial exp2, the rest the
-        // special-function unit.  P goes to tensor memory in two halves
-        // (keys 0-63, then 64-127); the MMA warp starts P V on the first half
-        // while the second is computed.
         const uint64_t sl2x2 = pack2(sl2, sl2);
         const uint64_t negm2 = pack2(-m, -m);
         uint64_t acc_a = pack2(0.f, 0.f), acc_b = pack2(0.f, 0.f);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-#pragma unroll
-          for (int c = 2 * half; c < 2 * half + 2; ++c) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const uint64_t x2 = ffma2(pack2(FA_S(c * 32 + 2 * e), FA_S(c * 32 + 2 * e + 1)), sl2x2, negm2);
-              uint64_t p2;
-              if ((C::POLY_MASK >> e) & 1u) {
-                p2 = exp2_poly2(x2);
-              } else {
-                float x0, x1;
-                unpack2(x2, x0, x1);
-                p2 = pack2(ex2_approx(x0), ex2_approx(x1));
-              }
-              if (e & 1)
-                acc_b = fadd2(acc_b, p2);
-              else
-                acc_a = fadd2(acc_a, p2);
-              float p0, p1;
-              unpack2(p2, p0, p1);
-              if constexpr (ELEM == kElemF16)
-                pk[e] = pack_f16x2(p0, p1);
-              else
-                pk[e] = pack_bf16x2(p0, p1);
-            }
-            tmem_st16(t_s + c * 16, pk);
+          exp_store_half<ELEM, C::POLY_MASK>(sr, half, sl2x2, negm2, t_s, acc_a, acc_b);
+          if (FA_SPLIT_P || half == 1) {
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b.p_full(wg, FA_SPLIT_P ? half : 0));
+            if (lane == 0 && wq == 0) FA_TRACE_EV(wg, 3 + half + 10 * wg, j);
           }
-          tmem_st_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(b.p_full(wg, half));
-          if (lane == 0 && wq == 0) FA_TRACE_EV(wg, 3 + half + 10 * wg, j);
         }
-#undef FA_S
-        {
-          float a0, a1, b0, b1;
-          unpack2(acc_a, a0, a1);
-          unpack2(acc_b, b0, b1);
-          l += (a0 + a1) + (b0 + b1);
-        }
+        l += sum_acc(acc_a, acc_b);
       }
       // epilogue: O / l -> global, LSE
       if (!wait_warp(o_full, o_cnt)) return false;
       ++o_cnt;
-      if (lane == 0 && wq == 0) FA_TRACE_EV(wg, 5 + 10 * wg, 0);
       tc_fence_after();
-      const float inv_l = 1.f / l;
-      OutT* orow = reinterpret_cast<OutT*>(a.o) + (static_cast<size_t>(t.bh) * a.N + qrow) * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t orr[32];
-        tmem_ld32(t_o + c * 32, orr);
-        tmem_ld_wait(orr);
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float v0 = __uint_as_float(orr[2 * e]) * inv_l;
-          const float v1 = __uint_as_float(orr[2 * e + 1]) * inv_l;
-          pk[e] = (ELEM == kElemF16) ? pack_f16x2(v0, v1) : pack_bf16x2(v0, v1);
-        }
-        if (qrow < a.N) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-        }
-      }
-      if (lane == 0 && wq == 0) FA_TRACE_EV(wg, 6 + 10 * wg, 0);
-      if (a.lse != nullptr && qrow < a.N)
-        a.lse[static_cast<size_t>(t.bh) * a.N + qrow] = (m + __log2f(l)) * 0.69314718055994531f;
+      epilogue_row<D, ELEM>(a, t_o, t.bh, qrow, m, l);
     }
     return true;
   };
   if (!run()) record_failure(a, abort_flag, kStatusSoftmax);
   tc_fence_before();
+}
+
+// Decoupled layout (d <= 64): S_i, P_i and O_i have separate tensor-memory
+// columns.  The warpgroup releases S_i right after loading it (s_free), so
+// the MMA issuer computes S_i(j+1) while this step's exponentials run, and it
+// writes P_i(j) only once P_i(j-1) V has completed (p_free), which also makes
+// O_i safe to rescale.
+template <int D, int ELEM>
+__device__ __forceinline__ void softmax_role_decoupled(const FwdArgs& a, const Bars<FwdCfg<D, ELEM>::NS> b,
+                                                       uint32_t tmem, int warp, int lane, volatile int* abort_flag) {
+  using C = FwdCfg<D, ELEM>;
+  const uint64_t limit = a.wait_limit_ns;
+  const int wg = warp >> 2;
+  const int wq = warp & 3;
+  const int row = wq * 32 + lane;
+  const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+  const uint32_t t_s = tmem + lane_off + (wg ? C::S_COL1 : C::S_COL0);
+  const uint32_t t_p = tmem + lane_off + (wg ? C::P_COL1 : C::P_COL0);
+  const uint32_t t_o = tmem + lane_off + (wg ? C::O_COL1 : C::O_COL0);
+  int s_cnt = 0, p_writes = 0, o_cnt = 0;
+  FA_TRACE_DECL;
+
+  auto wait_warp = [&](uint32_t bar, int parity) -> bool {
+    bool ok = wait_bounded(bar, parity & 1, abort_flag, limit);
+    return __all_sync(0xffffffffu, ok);
+  };
+  auto arrive_warp = [&](uint32_t bar) {
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar);
+  };
+
+  auto run = [&]() -> bool {
+    for (int w = blockIdx.x; w < a.n_work; w += gridDim.x) {
+      const WorkTile t = decode_work(a, w);
+      const int q_start = t.tp * 256 + wg * 128;
+      const int nkv = kv_tiles(a, q_start);
+      if (nkv == 0) continue;
+      const int qrow = q_start + row;
+      const float sl2 = a.scale_log2;
+      float m = -INFINITY;
+      float l = 0.f;
+      for (int j = 0; j < nkv; ++j) {
+        if (lane == 0 && wq == 0) FA_TRACE_EV(wg, 0 + 10 * wg, j);
+        if (!wait_warp(b.s_full(wg), s_cnt)) return false;
+        ++s_cnt;
+        tc_fence_after();
+        if (lane == 0 && wq == 0) FA_TRACE_EV(wg, 1 + 10 * wg, j);
+        uint32_t sr[4][32];
+        load_s_row(t_s, sr);
+        arrive_warp(b.s_free(wg));          // S_i may be overwritten now
+        if (lane == 0 && wq == 0) FA_TRACE_EV(wg, 2 + 10 * wg, j);
+        if (j == nkv - 1) mask_row(sr, j * 128, (a.causal && qrow < a.N - 1) ? qrow : a.N - 1);
+        const float mx = row_max(sr) * sl2;
+        bool rescale = false;
+        float alpha = 1.f;
+        if (j == 0) {
+          m = mx;
+        } else if (__any_sync(0xffffffffu, mx - m > C::TAU)) {
+          const float m_new = fmaxf(m, mx);
+          alpha = ex2_approx(m - m_new);
+          m = m_new;
+          l *= alpha;
+          rescale = true;
+        }
+        // exponentials into registers while P_i(j-1) V may still run
+        const uint64_t sl2x2 = pack2(sl2, sl2);
+        const uint64_t negm2 = pack2(-m, -m);
+        uint64_t acc_a = pack2(0.f, 0.f), acc_b = pack2(0.f, 0.f);
+        uint32_t pk[4][16];
+        exp_to_regs<ELEM, C::POLY_MASK>(sr, sl2x2, negm2, pk, acc_a, acc_b);
+        // the previous P_i V has read P_i and finished updating O_i
+        if (p_writes > 0) {
+          if (!wait_warp(b.p_free(wg), p_writes - 1)) return false;
+          tc_fence_after();
+        }
+        if (lane == 0 && wq == 0) FA_TRACE_EV(wg, 7 + 10 * wg, j);
+        if (rescale) rescale_o<D>(t_o, alpha);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_st16(t_p + c * 16, pk[c]);
+        tmem_st_wait();
+        arrive_warp(b.p_full(wg, 0));
+        if (lane == 0 && wq == 0) FA_TRACE_EV(wg, 4 + 10 * wg, j);
+        ++p_writes;
+        l += sum_acc(acc_a, acc_b);
+      }
+      if (!wait_warp(b.o_full(wg), o_cnt)) return false;
+      ++o_cnt;
+      tc_fence_after();
+      epilogue_row<D, ELEM>(a, t_o, t.bh, qrow, m, l);
+    }
+    return true;
+  };
+  if (!run()) record_failure(a, abort_flag, kStatusSoftmax);
+  tc_fence_before();
+}
+
+// ---------------------------------------------------------------- MMA (decoupled)
+// One issuer per Q tile (the tiles touch disjoint tensor memory and only
+// share the K/V ring).  Per step j: S_i(j+1) as soon as the softmax has
+// loaded S_i(j) and K_{j+1} is in, then P_i(j) V_j once P_i(j) is written.
+// A ring stage is released once both issuers are done with it (kv_empty
+// counts two arrivals); an issuer whose tile needs fewer K/V tiles (causal)
+// still releases the extra stages, after they are loaded, so the ring's
+// phases advance in step.
+template <int D, int ELEM>
+__device__ __forceinline__ void mma_role_decoupled(const FwdArgs& a, const Bars<FwdCfg<D, ELEM>::NS> b, const int i,
+                                                   uint32_t sQ_addr, uint32_t sKV_addr, uint32_t tmem,
+                                                   volatile int* abort_flag) {
+  using C = FwdCfg<D, ELEM>;
+  static_assert(ELEM != kElemE4M3, "the e4m3 path uses the aliased layout");
+  const uint64_t limit = a.wait_limit_ns;
+  const uint64_t dq = smem_desc(sQ_addr + i * C::Q_TILE, 16, 8 * C::SW_QK, C::SWZ_QK);
+  const uint64_t dkv0 = smem_desc(sKV_addr, 16, 8 * C::SW_QK, C::SWZ_QK);
+  const uint64_t dv0 = smem_desc(sKV_addr, C::BN * C::SW_V, 8 * C::SW_V, C::SWZ_V);
+  const uint32_t s_tmem = tmem + (i ? C::S_COL1 : C::S_COL0);
+  const uint32_t p_tmem = tmem + (i ? C::P_COL1 : C::P_COL0);
+  const uint32_t o_tmem = tmem + (i ? C::O_COL1 : C::O_COL0);
+  int pos = 0, q_use = 0, s_issued = 0, pv_issued = 0;
+  FA_TRACE_DECL;
+
+  auto acquire = [&](int p) -> int {
+    const int stage = p % C::NS;
+    if (!wait_bounded(b.kv_full(stage), (p / C::NS) & 1, abort_flag, limit)) return -1;
+    return stage;
+  };
+  // S_i = Q_i K^T into the S columns, once the softmax has read the last S_i
+  auto issue_s = [&](int stage) -> bool {
+    FA_TRACE_EV(2 + 4 * i, 44 + 2 * i, s_issued);
+    if (s_issued > 0 && !wait_bounded(b.s_free(i), (s_issued - 1) & 1, abort_flag, limit)) return false;
+    FA_TRACE_EV(2 + 4 * i, 45 + 2 * i, s_issued);
+    tc_fence_after();
+    const uint64_t ka = dkv0 + ((stage * C::STAGE) >> 4);
+#pragma unroll
+    for (int kk = 0; kk < C::K_STEPS_QK; ++kk) {
+      const uint32_t off = ((kk * 32) / C::SW_QK) * (C::BM * C::SW_QK) + ((kk * 32) % C::SW_QK);
+      mma_f16_ss(s_tmem, dq + (off >> 4), ka + (off >> 4), C::IDESC_QK, kk > 0);
+    }
+    tc_commit(b.s_full(i));
+    ++s_issued;
+    return true;
+  };
+  auto issue_pv = [&](int stage, bool accumulate) -> bool {
+    FA_TRACE_EV(2 + 4 * i, 30 + 2 * i, pv_issued);
+    if (!wait_bounded(b.p_full(i, 0), pv_issued & 1, abort_flag, limit)) return false;
+    FA_TRACE_EV(2 + 4 * i, 31 + 2 * i, pv_issued);
+    tc_fence_after();
+    const uint64_t va = dv0 + ((stage * C::STAGE) >> 4);
+#pragma unroll
+    for (int kk = 0; kk < C::K_STEPS_PV; ++kk)
+      mma_f16_ts(o_tmem, p_tmem + kk * 8, va + ((kk * 16 * C::SW_V) >> 4), C::IDESC_PV,
+                 (accumulate || kk > 0) ? 1u : 0u);
+    tc_commit(b.p_free(i));
+    ++pv_issued;
+    return true;
+  };
+
+  bool ok = true;
+  for (int w = blockIdx.x; ok && w < a.n_work; w += gridDim.x) {
+    const WorkTile t = decode_work(a, w);
+    const int q0 = t.tp * 256;
+    const int n0 = kv_tiles(a, q0), n1 = kv_tiles(a, q0 + 128);
+    const int nkv = n0 > n1 ? n0 : n1;
+    const int n = i ? n1 : n0;
+    if (n > 0) {
+      if (!wait_bounded(b.q_full(i), (q_use++) & 1, abort_flag, limit)) { ok = false; break; }
+      int sk = acquire(pos);
+      if (sk < 0 || !issue_s(sk)) { ok = false; break; }
+      if (n == 1) tc_commit(b.q_empty(i));
+      tc_commit(b.kv_empty(sk));
+      for (int j = 0; j < n; ++j) {
+        if (j + 1 < n) {
+          sk = acquire(pos + 2);
+          if (sk < 0 || !issue_s(sk)) { ok = false; break; }
+          if (j + 1 == n - 1) tc_commit(b.q_empty(i));
+          tc_commit(b.kv_empty(sk));
+        }
+        const int sv = acquire(pos + 1);
+        if (sv < 0 || !issue_pv(sv, j > 0)) { ok = false; break; }
+        if (j == n - 1) tc_commit(b.o_full(i));
+        tc_commit(b.kv_empty(sv));
+        pos += 2;
+      }
+      if (!ok) break;
+    }
+    // release-only for the K/V tiles of this work tile that tile i skips
+    for (int j = n; j < nkv && ok; ++j) {
+      for (int kind = 0; kind < 2; ++kind) {
+        const int st = acquire(pos + kind);
+        if (st < 0) { ok = false; break; }
+        mbar_arrive(b.kv_empty(st));
+      }
+      pos += 2;
+    }
+  }
+  if (!ok) record_failure(a, abort_flag, kStatusMma);
+  // Drain: all issued MMAs complete before tensor memory is released.
+  tc_commit(b.mma_done());
+  volatile int never = 0;
+  if (!wait_bounded(b.mma_done(), 0, &never, limit)) atomicOr(a.status, kStatusDrain);
 }
 
 template <int D, int ELEM>
@@ -608,9 +890,13 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(b.kv_full(s), 1);
-      mbar_init(b.kv_empty(s), 1);
+      mbar_init(b.kv_empty(s), C::ISSUERS);  // released by every MMA issuer
     }
-    mbar_init(b.mma_done(), 1);
+    mbar_init(b.mma_done(), C::ISSUERS);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(b.s_free(i), 4);
+      mbar_init(b.p_free(i), 1);
+    }
     fence_barrier_init();
   }
   if (warp == C::MMA_WARP) {
@@ -628,12 +914,21 @@ __global__ void __launch_bounds__(384, 1)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(C::REG_OTHER));
     if (warp == C::LOAD_WARP && lane == 0)
       producer_role<D, ELEM>(a, b, sQ, sKV, &map_q, &map_k, &map_v, abort_flag);
-    else if (warp == C::MMA_WARP && lane == 0)
-      mma_role<D, ELEM>(a, b, sQ, sKV, tmem, abort_flag);
-    // warps 10 and 11 only give their registers away
+    else if (lane == 0) {
+      if constexpr (C::DECOUPLED) {
+        if (warp == C::MMA_WARP || warp == C::MMA_WARP1)
+          mma_role_decoupled<D, ELEM>(a, b, warp == C::MMA_WARP ? 0 : 1, sQ, sKV, tmem, abort_flag);
+      } else {
+        if (warp == C::MMA_WARP) mma_role<D, ELEM>(a, b, sQ, sKV, tmem, abort_flag);
+      }
+    }
+    // the remaining warps of this warpgroup only give their registers away
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(C::REG_SOFTMAX));
-    softmax_role<D, ELEM>(a, b, tmem, warp, lane, abort_flag);
+    if constexpr (C::DECOUPLED)
+      softmax_role_decoupled<D, ELEM>(a, b, tmem, warp, lane, abort_flag);
+    else
+      softmax_role<D, ELEM>(a, b, tmem, warp, lane, abort_flag);
   }
 
   __syncthreads();
