@@ -158,8 +158,8 @@ fa_status fa_debug_withhold_arrival(int enable);
  *
  * The first call on a device does a one-time set-up with that device
  * current: it looks up the array's device address (cudaGetSymbolAddress) and
- * clears its status word with a synchronous cudaMemset.  Make that first call
- * before any stream capture.
+ * clears its status word and work-scheduling counters with a synchronous
+ * cudaMemset.  Make that first call before any stream capture.
  *
  * Every call on a device shares the one array, and the array keeps the last
  * call's contents.  Calls whose work overlaps on the GPU (different streams,
@@ -169,7 +169,7 @@ fa_status fa_debug_withhold_arrival(int enable);
  */
 #define FA_NOALLOC_MAX_ELEMS (8u * 1024u * 1024u)
 #define FA_NOALLOC_MAX_TILES (65536u)
-#define FA_NOALLOC_SCRATCH_BYTES (2u * FA_NOALLOC_MAX_ELEMS + 2u * 4u * FA_NOALLOC_MAX_TILES + 256u)
+#define FA_NOALLOC_SCRATCH_BYTES (2u * FA_NOALLOC_MAX_ELEMS + 2u * 4u * FA_NOALLOC_MAX_TILES + 256u + 2048u)
 fa_status fa_fwd_e4m3_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
                               int B, int H, int N, int d, float softmax_scale, int causal,
                               void* stream);

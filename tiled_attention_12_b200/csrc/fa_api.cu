@@ -7,6 +7,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -24,12 +25,18 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
 
 constexpr int kMaxDevices = 64;
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s
+// Scheduler counter pairs per device.  Each launch takes the next pair
+// round-robin; a pair is reset by the last CTA of the launch that used it, so
+// up to kSchedSlots launches may be in flight on one device at a time.
+constexpr int kSchedSlots = 256;
+constexpr size_t kScratchBytes = 256 + kSchedSlots * 2 * sizeof(unsigned int);
 
 struct DeviceState {
   bool ready = false;
   int sms = 0;
   int major = 0;
-  unsigned int* status = nullptr;  // device status word
+  unsigned int* status = nullptr;  // device status word, followed by the scheduler counters
+  std::atomic<unsigned> next_slot{0};
   void* ws = nullptr;              // FA_E4M3 workspace
   size_t ws_bytes = 0;
 };
@@ -57,8 +64,8 @@ fa_status device_state(DeviceState** out) {
     s.major = major;
     s.sms = sms;
     if (major != 10) return FA_ERR_ARCH;
-    if (cudaMalloc(&s.status, sizeof(unsigned int)) != cudaSuccess) return FA_ERR_CUDA;
-    if (cudaMemset(s.status, 0, sizeof(unsigned int)) != cudaSuccess) return FA_ERR_CUDA;
+    if (cudaMalloc(&s.status, kScratchBytes) != cudaSuccess) return FA_ERR_CUDA;
+    if (cudaMemset(s.status, 0, kScratchBytes) != cudaSuccess) return FA_ERR_CUDA;
     if (g_encode == nullptr) {
       void* fn = nullptr;
       cudaDriverEntryPointQueryResult q;
@@ -103,11 +110,15 @@ fa_status check_shape(int B, int H, int N, int d) {
 
 bool scale_ok(float s) { return std::isfinite(s) && s > 0.f; }
 
-// Causal schedule: heads per group so that about two waves of CTAs work on
-// the same few heads (their K/V stay in L2).
-int group_heads(int BH, int n_qpairs, int grid) {
-  int g = (2 * grid + n_qpairs - 1) / n_qpairs;
-  if (g < 1) g = 1;
+// Causal schedule: heads per group.  Inside a group the longest work tiles
+// go first; a group's K and V together should stay well inside the 126 MB
+// L2 (about 64 MiB), and groups of at least 4 heads keep the dynamic hand-out
+// balanced at the end of each group.
+int group_heads(int BH, int N, int d, int qk_bytes) {
+  const double kv_head = static_cast<double>(N) * d * (qk_bytes + 2);
+  int g = static_cast<int>((64.0 * 1024 * 1024) / kv_head);
+  if (g < 4) g = 4;
+  if (g > 16) g = 16;
   if (g > BH) g = BH;
   return g;
 }
@@ -129,6 +140,7 @@ fa_status launch_attention(DeviceState* ds, int elem, const void* q, const void*
   a.q_scale = q_scale;
   a.k_scale = k_scale;
   a.status = ds->status;
+  a.sched = ds->status + 64 + 2 * (ds->next_slot.fetch_add(1u) % kSchedSlots);
   a.BH = BH;
   a.N = N;
   a.n_qpairs = (N + 255) / 256;
@@ -143,7 +155,7 @@ fa_status launch_attention(DeviceState* ds, int elem, const void* q, const void*
     g_withhold = 0;
   }
   l.grid = a.n_work < ds->sms ? a.n_work : ds->sms;
-  a.group_heads = group_heads(BH, a.n_qpairs, l.grid);
+  a.group_heads = group_heads(BH, N, d, qk_bytes);
   l.args = &a;
   l.stream = stream;
   cudaError_t e;
@@ -265,7 +277,12 @@ fa_status fa_release(void) {
   DeviceState& s = g_dev[dev];
   if (s.ws) cudaFree(s.ws);
   if (s.status) cudaFree(s.status);
-  s = DeviceState();
+  s.ready = false;
+  s.sms = 0;
+  s.major = 0;
+  s.status = nullptr;
+  s.ws = nullptr;
+  s.ws_bytes = 0;
   return FA_OK;
 }
 

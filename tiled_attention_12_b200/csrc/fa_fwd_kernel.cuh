@@ -64,6 +64,7 @@ struct FwdArgs {
   const float* q_scale;    // [BH, ceil(N/128)] (e4m3 only)
   const float* k_scale;    // [BH, ceil(N/128)] (e4m3 only)
   unsigned int* status;    // device status word
+  unsigned int* sched;     // this launch's scheduler counters: [0] next work tile, [1] CTAs done
   int BH;                  // batch * heads
   int N;                   // sequence length
   int n_qpairs;            // ceil(N / 256): work tiles per head
@@ -95,7 +96,7 @@ struct FwdCfg {
   static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;  // K/V ring depth
   static_assert(NS >= 2, "ring too shallow");
   static constexpr int TILE_BYTES = 2 * Q_TILE + NS * STAGE;
-  static constexpr int NUM_BARS = 17 + 2 * NS;
+  static constexpr int NUM_BARS = 21 + 2 * NS;
   // at least 120 KB so that two CTAs never share an SM (each holds all 512
   // tensor-memory columns; a second resident CTA would only wait)
   static constexpr int SMEM_NEED = 1024 + TILE_BYTES + 8 * NUM_BARS;
@@ -162,7 +163,10 @@ struct Bars {
   // MMA that read P_i and updated O_i has completed
   __device__ __forceinline__ uint32_t s_free(int i) const { return base + 8u * (13 + 2 * NS + i); }
   __device__ __forceinline__ uint32_t p_free(int i) const { return base + 8u * (15 + 2 * NS + i); }
-  static constexpr int COUNT = 17 + 2 * NS;
+  // work-tile feed: the TMA thread publishes each tile index in a 2-slot ring
+  __device__ __forceinline__ uint32_t feed_full(int k) const { return base + 8u * (17 + 2 * NS + k); }
+  __device__ __forceinline__ uint32_t feed_empty(int k) const { return base + 8u * (19 + 2 * NS + k); }
+  static constexpr int COUNT = 21 + 2 * NS;
 };
 
 struct WorkTile {
@@ -208,6 +212,68 @@ __device__ __forceinline__ void record_failure(const FwdArgs& a, volatile int* a
   atomicOr(a.status, bit);
 }
 
+// Dynamic work distribution.  CTAs take work tiles in the order decode_work
+// defines (longest first, heads in L2-sized groups) from a per-launch global
+// counter, so each CTA picks up the next tile as soon as it is free.  The
+// TMA thread fetches the index and publishes it in a 2-slot shared-memory
+// ring; the MMA issuer(s) and the eight softmax warps each take it from
+// there and release the slot.  -1 ends the loop.
+struct TileFeed {
+  uint32_t full0, empty0;     // barrier addresses of slot 0 (slot 1 follows at +8)
+  volatile int* ring;         // [2]
+};
+
+template <int NS>
+__device__ __forceinline__ TileFeed make_feed(const Bars<NS>& b, volatile int* ring) {
+  return TileFeed{b.feed_full(0), b.feed_empty(0), ring};
+}
+
+__device__ __forceinline__ int feed_produce(const FwdArgs& a, const TileFeed& f, int& k, volatile int* abort_flag,
+                                            uint64_t limit, bool& ok) {
+  const int slot = k & 1;
+  if (k >= 2 && !wait_bounded(f.empty0 + 8u * slot, ((k >> 1) - 1) & 1, abort_flag, limit)) {
+    ok = false;
+    return -1;
+  }
+  int w = static_cast<int>(atomicAdd(a.sched, 1u));
+  if (w >= a.n_work) w = -1;
+  f.ring[slot] = w;
+  mbar_arrive(f.full0 + 8u * slot);
+  ++k;
+  return w;
+}
+
+// Single-thread consumer (an MMA issuer).
+__device__ __forceinline__ int feed_take(const TileFeed& f, int& k, volatile int* abort_flag, uint64_t limit,
+                                         bool& ok) {
+  const int slot = k & 1;
+  if (!wait_bounded(f.full0 + 8u * slot, (k >> 1) & 1, abort_flag, limit)) {
+    ok = false;
+    return -1;
+  }
+  const int w = f.ring[slot];
+  mbar_arrive(f.empty0 + 8u * slot);
+  ++k;
+  return w;
+}
+
+// Whole-warp consumer (a softmax warp): every lane gets the index, lane 0
+// releases the slot.
+__device__ __forceinline__ int feed_take_warp(const TileFeed& f, int& k, int lane, volatile int* abort_flag,
+                                              uint64_t limit, bool& ok) {
+  const int slot = k & 1;
+  const bool got = __all_sync(0xffffffffu, wait_bounded(f.full0 + 8u * slot, (k >> 1) & 1, abort_flag, limit));
+  if (!got) {
+    ok = false;
+    return -1;
+  }
+  const int w = f.ring[slot];
+  __syncwarp();
+  if (lane == 0) mbar_arrive(f.empty0 + 8u * slot);
+  ++k;
+  return w;
+}
+
 // ---------------------------------------------------------------- producer
 // One thread.  Per work tile: the Q tiles it needs, then K_j, V_j for every
 // K/V step into the ring.  Stage `it % NS` is reused in round `it / NS` once
@@ -215,7 +281,8 @@ __device__ __forceinline__ void record_failure(const FwdArgs& a, volatile int* a
 template <int D, int ELEM>
 __device__ __forceinline__ void producer_role(const FwdArgs& a, const Bars<FwdCfg<D, ELEM>::NS> b, uint32_t sQ,
                                               uint32_t sKV, const CUtensorMap* map_q, const CUtensorMap* map_k,
-                                              const CUtensorMap* map_v, volatile int* abort_flag) {
+                                              const CUtensorMap* map_v, const TileFeed feed,
+                                              volatile int* abort_flag) {
   using C = FwdCfg<D, ELEM>;
   const uint64_t limit = a.wait_limit_ns;
   tma_prefetch_desc(map_q);
@@ -225,7 +292,10 @@ __device__ __forceinline__ void producer_role(const FwdArgs& a, const Bars<FwdCf
   FA_TRACE_DECL;
   const bool withhold = a.withhold != 0;
   bool ok = true;
-  for (int w = blockIdx.x; ok && w < a.n_work; w += gridDim.x) {
+  int feed_k = 0;
+  while (ok) {
+    const int w = feed_produce(a, feed, feed_k, abort_flag, limit, ok);
+    if (w < 0) break;
     const WorkTile t = decode_work(a, w);
     const int q0 = t.tp * 256;
     const int n0 = kv_tiles(a, q0), n1 = kv_tiles(a, q0 + 128);
@@ -296,7 +366,8 @@ __device__ __forceinline__ void producer_role(const FwdArgs& a, const Bars<FwdCf
 // field, which cannot overflow for shared-memory addresses below 256 KB.
 template <int D, int ELEM>
 __device__ __forceinline__ void mma_role(const FwdArgs& a, const Bars<FwdCfg<D, ELEM>::NS> b, uint32_t sQ_addr,
-                                         uint32_t sKV_addr, uint32_t tmem, volatile int* abort_flag) {
+                                         uint32_t sKV_addr, uint32_t tmem, const TileFeed feed,
+                                         volatile int* abort_flag) {
   using C = FwdCfg<D, ELEM>;
   const uint64_t limit = a.wait_limit_ns;
   const uint64_t dq0 = smem_desc(sQ_addr, 16, 8 * C::SW_QK, C::SWZ_QK);
@@ -347,7 +418,10 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const Bars<FwdCfg<D, 
   };
 
   bool ok = true;
-  for (int w = blockIdx.x; ok && w < a.n_work; w += gridDim.x) {
+  int feed_k = 0;
+  while (ok) {
+    const int w = feed_take(feed, feed_k, abort_flag, limit, ok);
+    if (w < 0) break;
     const WorkTile t = decode_work(a, w);
     const int q0 = t.tp * 256;
     const int n0 = kv_tiles(a, q0), n1 = kv_tiles(a, q0 + 128);
@@ -580,7 +654,7 @@ __device__ __forceinline__ void epilogue_row(const FwdArgs& a, uint32_t t_o, int
 // MMA warp's order (S_i(j+1) after P_i(j) V) sequences the reuse.
 template <int D, int ELEM>
 __device__ __forceinline__ void softmax_role(const FwdArgs& a, const Bars<FwdCfg<D, ELEM>::NS> b, uint32_t tmem,
-                                             int warp, int lane, volatile int* abort_flag) {
+                                             int warp, int lane, const TileFeed feed, volatile int* abort_flag) {
   using C = FwdCfg<D, ELEM>;
   const uint64_t limit = a.wait_limit_ns;
   const int wg = warp >> 2;            // which Q tile
@@ -600,7 +674,12 @@ __device__ __forceinline__ void softmax_role(const FwdArgs& a, const Bars<FwdCfg
   };
 
   auto run = [&]() -> bool {
-    for (int w = blockIdx.x; w < a.n_work; w += gridDim.x) {
+    int feed_k = 0;
+    while (true) {
+      bool fed = true;
+      const int w = feed_take_warp(feed, feed_k, lane, abort_flag, limit, fed);
+      if (!fed) return false;
+      if (w < 0) break;
       const WorkTile t = decode_work(a, w);
       const int q_start = t.tp * 256 + wg * 128;
       const int nkv = kv_tiles(a, q_start);
@@ -667,7 +746,8 @@ __device__ __forceinline__ void softmax_role(const FwdArgs& a, const Bars<FwdCfg
 // O_i safe to rescale.
 template <int D, int ELEM>
 __device__ __forceinline__ void softmax_role_decoupled(const FwdArgs& a, const Bars<FwdCfg<D, ELEM>::NS> b,
-                                                       uint32_t tmem, int warp, int lane, volatile int* abort_flag) {
+                                                       uint32_t tmem, int warp, int lane, const TileFeed feed,
+                                                       volatile int* abort_flag) {
   using C = FwdCfg<D, ELEM>;
   const uint64_t limit = a.wait_limit_ns;
   const int wg = warp >> 2;
@@ -691,7 +771,12 @@ __device__ __forceinline__ void softmax_role_decoupled(const FwdArgs& a, const B
   };
 
   auto run = [&]() -> bool {
-    for (int w = blockIdx.x; w < a.n_work; w += gridDim.x) {
+    int feed_k = 0;
+    while (true) {
+      bool fed = true;
+      const int w = feed_take_warp(feed, feed_k, lane, abort_flag, limit, fed);
+      if (!fed) return false;
+      if (w < 0) break;
       const WorkTile t = decode_work(a, w);
       const int q_start = t.tp * 256 + wg * 128;
       const int nkv = kv_tiles(a, q_start);
@@ -766,7 +851,7 @@ __device__ __forceinline__ void softmax_role_decoupled(const FwdArgs& a, const B
 template <int D, int ELEM>
 __device__ __forceinline__ void mma_role_decoupled(const FwdArgs& a, const Bars<FwdCfg<D, ELEM>::NS> b, const int i,
                                                    uint32_t sQ_addr, uint32_t sKV_addr, uint32_t tmem,
-                                                   volatile int* abort_flag) {
+                                                   const TileFeed feed, volatile int* abort_flag) {
   using C = FwdCfg<D, ELEM>;
   static_assert(ELEM != kElemE4M3, "the e4m3 path uses the aliased layout");
   const uint64_t limit = a.wait_limit_ns;
@@ -816,7 +901,10 @@ __device__ __forceinline__ void mma_role_decoupled(const FwdArgs& a, const Bars<
   };
 
   bool ok = true;
-  for (int w = blockIdx.x; ok && w < a.n_work; w += gridDim.x) {
+  int feed_k = 0;
+  while (ok) {
+    const int w = feed_take(feed, feed_k, abort_flag, limit, ok);
+    if (w < 0) break;
     const WorkTile t = decode_work(a, w);
     const int q0 = t.tp * 256;
     const int n0 = kv_tiles(a, q0), n1 = kv_tiles(a, q0 + 128);
@@ -868,6 +956,7 @@ __global__ void __launch_bounds__(384, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t tmem_holder;
   __shared__ int abort_flag_storage;
+  __shared__ int feed_ring[2];
   volatile int* abort_flag = &abort_flag_storage;
 
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -893,6 +982,10 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(b.kv_empty(s), C::ISSUERS);  // released by every MMA issuer
     }
     mbar_init(b.mma_done(), C::ISSUERS);
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(b.feed_full(k), 1);
+      mbar_init(b.feed_empty(k), C::ISSUERS + 8);  // MMA issuer(s) and the eight softmax warps
+    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(b.s_free(i), 4);
       mbar_init(b.p_free(i), 1);
@@ -907,34 +1000,44 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_holder;
+  const TileFeed feed = make_feed(b, feed_ring);
 
   // Each role's code sits inside the branch that set its register budget, so
   // the compiler allocates the softmax code for REG_SOFTMAX registers.
   if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(C::REG_OTHER));
     if (warp == C::LOAD_WARP && lane == 0)
-      producer_role<D, ELEM>(a, b, sQ, sKV, &map_q, &map_k, &map_v, abort_flag);
+      producer_role<D, ELEM>(a, b, sQ, sKV, &map_q, &map_k, &map_v, feed, abort_flag);
     else if (lane == 0) {
       if constexpr (C::DECOUPLED) {
         if (warp == C::MMA_WARP || warp == C::MMA_WARP1)
-          mma_role_decoupled<D, ELEM>(a, b, warp == C::MMA_WARP ? 0 : 1, sQ, sKV, tmem, abort_flag);
+          mma_role_decoupled<D, ELEM>(a, b, warp == C::MMA_WARP ? 0 : 1, sQ, sKV, tmem, feed, abort_flag);
       } else {
-        if (warp == C::MMA_WARP) mma_role<D, ELEM>(a, b, sQ, sKV, tmem, abort_flag);
+        if (warp == C::MMA_WARP) mma_role<D, ELEM>(a, b, sQ, sKV, tmem, feed, abort_flag);
       }
     }
     // the remaining warps of this warpgroup only give their registers away
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(C::REG_SOFTMAX));
     if constexpr (C::DECOUPLED)
-      softmax_role_decoupled<D, ELEM>(a, b, tmem, warp, lane, abort_flag);
+      softmax_role_decoupled<D, ELEM>(a, b, tmem, warp, lane, feed, abort_flag);
     else
-      softmax_role<D, ELEM>(a, b, tmem, warp, lane, abort_flag);
+      softmax_role<D, ELEM>(a, b, tmem, warp, lane, feed, abort_flag);
   }
 
   __syncthreads();
   if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+  // The last CTA to finish resets this launch's scheduler counters; every
+  // other CTA has made its final fetch by then.
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(a.sched + 1, 1u) == gridDim.x - 1) {
+      atomicExch(a.sched, 0u);
+      atomicExch(a.sched + 1, 0u);
+    }
   }
 }
 

@@ -35,10 +35,13 @@ constexpr size_t kMaxTiles = FA_NOALLOC_MAX_TILES;   // per operand (scales)
 constexpr size_t kCodesBytes = kMaxElems;            // one byte per e4m3 code
 constexpr size_t kScalesBytes = kMaxTiles * sizeof(float);
 constexpr size_t kStatusOffset = 2 * kCodesBytes + 2 * kScalesBytes;
-constexpr size_t kScratchBytes = kStatusOffset + 256;
+constexpr int kSchedSlots = 256;                     // scheduler counter pairs (see fa_api.cu)
+constexpr size_t kSchedOffset = kStatusOffset + 256;
+constexpr size_t kScratchBytes = kSchedOffset + kSchedSlots * 2 * sizeof(unsigned int);
 static_assert(kScratchBytes == FA_NOALLOC_SCRATCH_BYTES, "header and implementation disagree");
 
-// Layout: [q codes | k codes | q scales | k scales | status word (+pad)].
+// Layout: [q codes | k codes | q scales | k scales | status word (+pad) |
+// scheduler counters].
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -49,6 +52,7 @@ struct NoAllocDevice {
   bool ready = false;
   int sms = 0;
   unsigned char* scratch = nullptr;  // device address of g_noalloc_scratch on this device
+  unsigned next_slot = 0;            // guarded by g_na_mu
 };
 
 constexpr int kMaxDevices = 64;
@@ -70,7 +74,7 @@ fa_status noalloc_setup(NoAllocDevice** out) {
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FA_ERR_CUDA;
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return FA_ERR_CUDA;
-    if (cudaMemset(static_cast<unsigned char*>(ptr) + kStatusOffset, 0, sizeof(unsigned int)) != cudaSuccess)
+    if (cudaMemset(static_cast<unsigned char*>(ptr) + kStatusOffset, 0, kScratchBytes - kStatusOffset) != cudaSuccess)
       return FA_ERR_CUDA;
     if (g_na_encode == nullptr) {
       void* fn = nullptr;
@@ -149,6 +153,10 @@ extern "C" fa_status fa_fwd_e4m3_noalloc(const void* q, const void* k, const voi
   a.q_scale = qs;
   a.k_scale = ks;
   a.status = status;
+  {
+    std::lock_guard<std::mutex> lock(g_na_mu);
+    a.sched = reinterpret_cast<unsigned int*>(dev->scratch + kSchedOffset) + 2 * (dev->next_slot++ % kSchedSlots);
+  }
   a.BH = bh;
   a.N = N;
   a.n_qpairs = (N + 255) / 256;
@@ -159,8 +167,11 @@ extern "C" fa_status fa_fwd_e4m3_noalloc(const void* q, const void* k, const voi
   a.wait_limit_ns = 2000000000ull;
   a.withhold = 0;
   l.grid = a.n_work < dev->sms ? a.n_work : dev->sms;
-  int g = (2 * l.grid + a.n_qpairs - 1) / a.n_qpairs;
-  a.group_heads = g < 1 ? 1 : (g > bh ? bh : g);
+  // heads per causal scheduling group, as in fa_fwd: a group's K and V stay
+  // within about 64 MiB of L2, 4 to 16 heads
+  int g = static_cast<int>((64.0 * 1024 * 1024) / (static_cast<double>(N) * d * 3));
+  g = g < 4 ? 4 : (g > 16 ? 16 : g);
+  a.group_heads = g > bh ? bh : g;
   l.args = &a;
   l.stream = s;
   return fa::launch_fwd_e4m3(d, l) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
