@@ -1,0 +1,95 @@
+"""Per-configuration report: GPU time, TFLOPS, and parity errors against the
+fp64 oracle (all rows for small cases, sampled rows for large ones).
+
+    python tests/parity_report.py            # needs the GPU; prints a markdown table
+
+Not collected by pytest (no test_ prefix); the tests enforce the tolerances,
+this script only reports the measured errors.
+"""
+
+from __future__ import annotations
+
+import os
+import statistics
+import sys
+import time
+
+import numpy as np
+import torch
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+
+import tiled_attention_12_b200 as fa  # noqa: E402
+from oracle import (attention_ref, attention_rows, dequantize_e4m3_tiles,  # noqa: E402
+                    quantize_e4m3_tiles)
+from parity_util import half_ulp, sample_rows  # noqa: E402
+from tiled_attention_12_b200.synth import WORKLOADS, make_qkv  # noqa: E402
+
+PEAK_MEASURED = 1672.3
+PEAK_DATASHEET = 2250.0
+
+
+def gpu_time(fn, reps=10):
+    flush = torch.empty(128 << 20, device="cuda", dtype=torch.float32)
+    for _ in range(3):
+        fn()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(True), torch.cuda.Event(True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def main():
+    print("| case | GPU ms | TFLOPS | % datasheet | % measured | oracle rows | max-abs | max-abs − ½ulp | mean-abs | LSE max-abs | oracle s |")
+    print("|---|---|---|---|---|---|---|---|---|---|---|")
+    for wname, w in WORKLOADS.items():
+        for c in w.cases:
+            q, k, v = make_qkv(c)
+            qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+            dtype = fa.FA_E4M3 if c.fp8 else None
+            o, lse = fa.fa_fwd(qd, kd, vd, causal=c.causal, dtype=dtype)
+            torch.cuda.synchronize()
+            assert fa.fa_last_device_status() == 0
+            ms = gpu_time(lambda: fa.fa_fwd(qd, kd, vd, o=o, lse=lse, causal=c.causal, dtype=dtype))
+            tf = c.flops / ms / 1e9
+            if c.fp8:
+                cq, sq = quantize_e4m3_tiles(q)
+                ck, sk = quantize_e4m3_tiles(k)
+                q_ref, k_ref = dequantize_e4m3_tiles(cq, sq), dequantize_e4m3_tiles(ck, sk)
+            else:
+                q_ref, k_ref = q, k
+            t0 = time.perf_counter()
+            errs = []
+            if c.flops <= 2e10:
+                o_ref, lse_ref = attention_ref(q_ref, k_ref, v, c.softmax_scale, c.causal)
+                pairs = [(o.float().cpu().double().numpy(), o_ref, lse.cpu().double().numpy(), lse_ref)]
+                nrows = "all"
+            else:
+                pairs = []
+                oc, lc = o.float().cpu().double().numpy(), lse.cpu().double().numpy()
+                heads = sorted({(0, 0), (c.B - 1, c.H - 1), (c.B // 2, c.H // 2)})
+                n = 0
+                for b, h in heads:
+                    rows = sample_rows(c.N, seed=b * 1000 + h)
+                    o_r, l_r = attention_rows(q_ref, k_ref, v, c.softmax_scale, c.causal, b, h, rows)
+                    pairs.append((oc[b, h][rows], o_r, lc[b, h][rows], l_r))
+                    n += len(rows)
+                nrows = f"{n} sampled"
+            t_or = time.perf_counter() - t0
+            err = np.concatenate([np.abs(g - r).ravel() for g, r, _, _ in pairs])
+            exc = np.concatenate([np.maximum(0, np.abs(g - r) - half_ulp(r, torch.bfloat16)).ravel() for g, r, _, _ in pairs])
+            lerr = np.concatenate([np.abs(g - r).ravel() for _, _, g, r in pairs])
+            print(f"| {c.name} | {ms:.4f} | {tf:.1f} | {100 * tf / PEAK_DATASHEET:.1f} | {100 * tf / PEAK_MEASURED:.1f} | "
+                  f"{nrows} | {err.max():.2e} | {exc.max():.2e} | {err.mean():.2e} | {lerr.max():.2e} | {t_or:.1f} |",
+                  flush=True)
+
+
+if __name__ == "__main__":
+    main()
