@@ -141,6 +141,7 @@ def run_ours(args, rank, world, local_rank):
     import torch
 
     import tiled_attention_12_b200 as fa
+    from tiled_attention_12_b200.dist import aggregate_throughput, max_over_ranks
     from tiled_attention_12_b200.synth import WORKLOADS
 
     torch.cuda.set_device(local_rank)
@@ -218,13 +219,9 @@ def run_ours(args, rank, world, local_rank):
         raise SystemExit(f"device status {status} after the timed region")
     per_case_ms = [[ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(args.steps)] for i in range(n_cases)]
     total_ms = sum(sum(x) for x in per_case_ms)
-    t_max = total_ms
-    if dist is not None:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_max = float(t.item())
+    t_max = max_over_ranks(total_ms, device=dev)
     flops_step = sum(c.flops for c in cases)
-    value = world * flops_step * args.steps / (t_max * 1e-3) / 1e12
+    value = aggregate_throughput(flops_step, args.steps, world, t_max)
 
     result = {"flops_step": flops_step, "t_ms": t_max, "value": value, "clocks": clocks,
               "per_case_ms": per_case_ms}
@@ -269,12 +266,8 @@ def run_ours(args, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        e2e_ms = e0.elapsed_time(e1)
-        if dist is not None:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        result["e2e"] = {"value": round(world * flops_step * k_e2e / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOPS",
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), device=dev)
+        result["e2e"] = {"value": round(aggregate_throughput(flops_step, k_e2e, world, e2e_ms), 3), "unit": "TFLOPS",
                          "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k_e2e}
 
     # ---- per-workload suite (rank 0 only, single GPU numbers)
