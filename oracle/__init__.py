@@ -26,9 +26,10 @@ from .online import online_attention
 from .brute import brute_attention
 from .e4m3 import e4m3_decode, e4m3_encode_rne_satfinite, E4M3_MAX
 from .quantize import quantize_e4m3_tiles, dequantize_e4m3_tiles
+from .backward import attention_bwd_ref, attention_bwd_d
 
 __all__ = [
     "attention_ref", "attention_rows", "attention_flops", "online_attention",
     "brute_attention", "e4m3_decode", "e4m3_encode_rne_satfinite", "E4M3_MAX",
-    "quantize_e4m3_tiles", "dequantize_e4m3_tiles",
+    "quantize_e4m3_tiles", "dequantize_e4m3_tiles", "attention_bwd_ref", "attention_bwd_d",
 ]
