@@ -103,6 +103,25 @@ fa_status fa_fwd_fp8(const void* q8, const float* q_scale, const void* k8, const
                      float softmax_scale, int causal, void* stream);
 
 /*
+ * fa_bwd — gradients of fa_fwd by recomputation ("从理论到实现…" §2.2: no
+ * intermediate is stored; S and P are recomputed from Q, K and the forward's
+ * LSE).  With P = exp(softmax_scale * Q K^T - LSE) (causal mask as in fa_fwd):
+ *     dV = P^T dO,  dS = P * (dO V^T - rowsum(dO * O)),
+ *     dQ = softmax_scale * dS K,  dK = softmax_scale * dS^T Q.
+ *   q, k, v, o, dout : [B, H, N, d] bf16 or fp16 (per dtype; FA_E4M3 is not
+ *                      supported here); o and lse are fa_fwd's outputs for
+ *                      these q, k, v.
+ *   lse              : [B, H, N] fp32, natural log.
+ *   dq, dk, dv       : [B, H, N, d] outputs in the input element type; must
+ *                      not alias any input or each other.
+ * The library keeps a [B, H, N] fp32 workspace for rowsum(dO * O), grown on
+ * demand with cudaMalloc and freed by fa_release.
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                 float softmax_scale, int causal, fa_dtype dtype, void* stream);
+
+/*
  * fa_last_device_status — synchronises `stream`, reads and clears the device
  * status word of the current device.  FA_OK when no kernel on this device
  * gave up on a wait since the last call; FA_ERR_TIMEOUT otherwise.

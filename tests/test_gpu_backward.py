@@ -1,0 +1,79 @@
+"""GPU parity of the backward pass (fa_bwd) against the fp64 oracle."""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import tiled_attention_12_b200 as fa
+from oracle import attention_bwd_ref
+from tiled_attention_12_b200.synth import Case, make_qkv, make_tensor
+
+pytestmark = pytest.mark.gpu
+
+# Relative tolerances on each gradient: the kernel rounds P and dS to the
+# 16-bit input type before the accumulating products (relative 2^-9 per
+# element, random in sign, summed over up to N terms) and stores the result
+# in 16 bits; 2 % of the gradient's largest entry bounds the worst element
+# and 0.5 % of its mean magnitude bounds the mean error.  The absolute floor
+# covers gradients that are exactly zero (one key: dS = dP - D = 0), where the
+# kernel returns fp32 rounding noise.
+TOL_MAX_REL = 2e-2
+TOL_MEAN_REL = 5e-3
+TOL_ABS = 1e-4
+
+
+def _check(name, g, ref):
+    g = g.float().cpu().double().numpy()
+    err = np.abs(g - ref)
+    scale_max = np.abs(ref).max()
+    scale_mean = np.abs(ref).mean()
+    assert np.all(np.isfinite(g)), name
+    assert err.max() <= TOL_MAX_REL * scale_max + TOL_ABS, (name, err.max(), scale_max)
+    assert err.mean() <= TOL_MEAN_REL * scale_mean + TOL_ABS, (name, err.mean(), scale_mean)
+    return err.max() / max(scale_max, 1e-30), err.mean() / max(scale_mean, 1e-30)
+
+
+def _run(case: Case, dtype=torch.bfloat16):
+    q, k, v = make_qkv(case, dtype=dtype)
+    g = make_tensor((case.B, case.H, case.N, case.d), case.seed + 77, dtype=dtype)
+    qd, kd, vd, gd = q.cuda(), k.cuda(), v.cuda(), g.cuda()
+    o, lse = fa.fa_fwd(qd, kd, vd, causal=case.causal)
+    dq, dk, dv = fa.fa_bwd(qd, kd, vd, o, lse, gd, causal=case.causal)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status() == 0
+    rq, rk, rv = attention_bwd_ref(q, k, v, g, case.softmax_scale, case.causal)
+    return [_check("dq", dq, rq), _check("dk", dk, rk), _check("dv", dv, rv)]
+
+
+SHAPES = [(1, 2, n, d) for n in (1, 100, 128, 257, 300, 640) for d in (32, 64, 128)]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_backward_small(shape, causal):
+    B, H, N, d = shape
+    _run(Case("bwd", B, H, N, d, causal, seed=N + d))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_fp16(causal):
+    _run(Case("bwd16", 2, 2, 333, 64, causal, seed=5), dtype=torch.float16)
+
+
+def test_backward_many_heads_and_blocks():
+    _run(Case("bwdbig", 2, 8, 1024, 128, True, seed=6, value_scale=0.5))
+
+
+def test_backward_rejects_fp8_and_aliasing():
+    c = Case("x", 1, 1, 128, 128, False, seed=1)
+    q, k, v = (t.cuda() for t in make_qkv(c))
+    o, lse = fa.fa_fwd(q, k, v)
+    L = fa.load()
+    s = torch.cuda.current_stream().cuda_stream
+    p = [t.data_ptr() for t in (q, k, v, o, q, lse)]
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    assert L.fa_bwd(*p, dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), 1, 1, 128, 128, 0.1, 0, 2, s) == 2
+    assert L.fa_bwd(*p, q.data_ptr(), dk.data_ptr(), dv.data_ptr(), 1, 1, 128, 128, 0.1, 0, 0, s) == 1
+    assert L.fa_bwd(*p, dq.data_ptr(), dq.data_ptr(), dv.data_ptr(), 1, 1, 128, 128, 0.1, 0, 0, s) == 1

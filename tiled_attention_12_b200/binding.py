@@ -47,13 +47,14 @@ def load():
     L.fa_quantize_e4m3.argtypes = [vp, vp, vp, i, i, i, i, vp]
     L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     L.fa_fwd_e4m3_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
     L.fa_last_device_status.argtypes = [vp]
     L.fa_status_string.argtypes = [i]
     L.fa_status_string.restype = ctypes.c_char_p
     L.fa_release.argtypes = []
     L.fa_debug_set_wait_limit.argtypes = [ctypes.c_uint64]
     L.fa_debug_withhold_arrival.argtypes = [i]
-    for name in ("fa_fwd", "fa_quantize_e4m3", "fa_fwd_fp8", "fa_fwd_e4m3_noalloc", "fa_last_device_status",
+    for name in ("fa_fwd", "fa_bwd", "fa_quantize_e4m3", "fa_fwd_fp8", "fa_fwd_e4m3_noalloc", "fa_last_device_status",
                  "fa_release",
                  "fa_debug_set_wait_limit", "fa_debug_withhold_arrival"):
         getattr(L, name).restype = ctypes.c_int
@@ -115,6 +116,24 @@ def fa_fwd(q, k, v, o=None, lse=None, softmax_scale=None, causal=False, dtype=No
                        int(bool(causal)), code, _stream(stream))
     _check(st, "fa_fwd")
     return o, lse
+
+
+def fa_bwd(q, k, v, o, lse, dout, dq=None, dk=None, dv=None, softmax_scale=None, causal=False, stream=None):
+    """Gradients (dq, dk, dv) of fa_fwd for upstream dout, from fa_fwd's o and lse."""
+    import torch
+
+    for t in (q, k, v, o, dout):
+        if not (t.is_cuda and t.is_contiguous() and t.shape == q.shape and t.dtype == q.dtype):
+            raise ValueError("q, k, v, o, dout must be contiguous CUDA tensors of one shape and dtype")
+    B, H, N, d = q.shape
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    scale = (1.0 / d ** 0.5) if softmax_scale is None else float(softmax_scale)
+    st = load().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                       B, H, N, d, scale, int(bool(causal)), _dtype_code(q), _stream(stream))
+    _check(st, "fa_bwd")
+    return dq, dk, dv
 
 
 def fa_quantize_e4m3(x, x8=None, scales=None, stream=None):

@@ -14,6 +14,7 @@
 #include <mutex>
 
 #include "fa.h"
+#include "fa_bwd_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
 #include "fa_launch.h"
 
@@ -39,6 +40,8 @@ struct DeviceState {
   std::atomic<unsigned> next_slot{0};
   void* ws = nullptr;              // FA_E4M3 workspace
   size_t ws_bytes = 0;
+  float* bwd_ws = nullptr;         // backward: D = rowsum(dO * O)
+  size_t bwd_ws_bytes = 0;
 };
 
 std::mutex g_mu;
@@ -246,6 +249,67 @@ fa_status fa_fwd_fp8(const void* q8, const float* q_scale, const void* k8, const
                           causal, static_cast<cudaStream_t>(stream));
 }
 
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                 void* dq, void* dk, void* dv, int B, int H, int N, int d, float softmax_scale, int causal,
+                 fa_dtype dtype, void* stream) {
+  if (dtype != FA_BF16 && dtype != FA_FP16 && dtype != FA_E4M3) return FA_ERR_INVALID;
+  fa_status st = check_shape(B, H, N, d);
+  if (st != FA_OK) return st;
+  if (dtype == FA_E4M3) return FA_ERR_UNSUPPORTED;
+  const void* ins[6] = {q, k, v, o, dout, lse};
+  void* outs[3] = {dq, dk, dv};
+  for (const void* p : ins)
+    if (!p || !aligned16(p)) return FA_ERR_INVALID;
+  for (void* p : outs) {
+    if (!p || !aligned16(p)) return FA_ERR_INVALID;
+    for (const void* in : ins)
+      if (p == in) return FA_ERR_INVALID;
+  }
+  if (dq == dk || dq == dv || dk == dv) return FA_ERR_INVALID;
+  if (!scale_ok(softmax_scale) || (causal != 0 && causal != 1)) return FA_ERR_INVALID;
+
+  DeviceState* ds = nullptr;
+  if ((st = device_state(&ds)) != FA_OK) return st;
+  const int BH = B * H;
+  const size_t need = static_cast<size_t>(BH) * N * sizeof(float);
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (ds->bwd_ws_bytes < need) {
+      if (ds->bwd_ws) cudaFree(ds->bwd_ws);
+      ds->bwd_ws = nullptr;
+      ds->bwd_ws_bytes = 0;
+      if (cudaMalloc(&ds->bwd_ws, need) != cudaSuccess) return FA_ERR_CUDA;
+      ds->bwd_ws_bytes = need;
+    }
+  }
+  const bool fp16 = dtype == FA_FP16;
+  fa::BwdLaunch l;
+  if ((st = make_map(&l.map_q, q, BH, N, d, 2, fp16)) != FA_OK) return st;
+  if ((st = make_map(&l.map_k, k, BH, N, d, 2, fp16)) != FA_OK) return st;
+  if ((st = make_map(&l.map_v, v, BH, N, d, 2, fp16)) != FA_OK) return st;
+  if ((st = make_map(&l.map_do, dout, BH, N, d, 2, fp16)) != FA_OK) return st;
+  fa::BwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.o = o;
+  a.dout = dout;
+  a.lse = lse;
+  a.delta = ds->bwd_ws;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.status = ds->status;
+  a.BH = BH;
+  a.N = N;
+  a.causal = causal;
+  a.nblk = (N + 127) / 128;
+  a.scale = softmax_scale;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.wait_limit_ns = g_wait_ns;
+  l.args = &a;
+  l.stream = static_cast<cudaStream_t>(stream);
+  return map_cuda(fa::launch_bwd(d, fp16 ? fa::kElemF16 : fa::kElemBF16, l));
+}
+
 fa_status fa_last_device_status(void* stream) {
   DeviceState* ds = nullptr;
   fa_status st = device_state(&ds);
@@ -276,6 +340,7 @@ fa_status fa_release(void) {
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState& s = g_dev[dev];
   if (s.ws) cudaFree(s.ws);
+  if (s.bwd_ws) cudaFree(s.bwd_ws);
   if (s.status) cudaFree(s.status);
   s.ready = false;
   s.sms = 0;
@@ -283,6 +348,8 @@ fa_status fa_release(void) {
   s.status = nullptr;
   s.ws = nullptr;
   s.ws_bytes = 0;
+  s.bwd_ws = nullptr;
+  s.bwd_ws_bytes = 0;
   return FA_OK;
 }
 

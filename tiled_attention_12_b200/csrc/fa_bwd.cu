@@ -1,0 +1,49 @@
+// fa_bwd.cu — instantiations and launches of the backward kernels.
+#include "fa_bwd_kernel.cuh"
+#include "fa_launch.h"
+
+namespace fa {
+
+namespace {
+
+template <int D, int ELEM>
+cudaError_t launch_bwd_t(const BwdLaunch& l) {
+  using C = BwdCfg<D, ELEM>;
+  const BwdArgs& a = *l.args;
+  const long long rows = static_cast<long long>(a.BH) * a.N;
+  bwd_d_kernel<D, ELEM><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, l.stream>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>(a.BH) * static_cast<unsigned>(a.nblk);
+  auto kdkdv = fa_bwd_dkdv_kernel<D, ELEM>;
+  auto kdq = fa_bwd_dq_kernel<D, ELEM>;
+  if ((e = cudaFuncSetAttribute(kdkdv, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)) != cudaSuccess)
+    return e;
+  kdkdv<<<grid, 192, C::SMEM_BYTES, l.stream>>>(l.map_q, l.map_k, l.map_v, l.map_do, a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  kdq<<<grid, 192, C::SMEM_BYTES, l.stream>>>(l.map_q, l.map_k, l.map_v, l.map_do, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd(int d, int elem, const BwdLaunch& l) {
+  if (elem == kBwdElemF16) {
+    switch (d) {
+      case 32: return launch_bwd_t<32, kBwdElemF16>(l);
+      case 64: return launch_bwd_t<64, kBwdElemF16>(l);
+      case 128: return launch_bwd_t<128, kBwdElemF16>(l);
+    }
+  } else {
+    switch (d) {
+      case 32: return launch_bwd_t<32, kBwdElemBF16>(l);
+      case 64: return launch_bwd_t<64, kBwdElemBF16>(l);
+      case 128: return launch_bwd_t<128, kBwdElemBF16>(l);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace fa

@@ -1,0 +1,525 @@
+// fa_bwd_kernel.cuh — attention backward by recomputation for sm_100a.
+//
+// No intermediate of the forward is stored; S and P are recomputed from Q,
+// K and the forward's per-row log-sum-exp ("从理论到实现：基于Triton剖析
+// FlashAttention三代的演进与优化" §2.2, 重计算机制).  With S = scale * Q K^T:
+//
+//     P = exp(S - LSE),  dV = P^T dO,  dP = dO V^T,  D = rowsum(dO * O),
+//     dS = P * (dP - D), dQ = scale * dS K,  dK = scale * dS^T Q.
+//
+// Three kernels:
+//   bwd_d_kernel       D = rowsum(dO * O), one warp per row (HBM-bound).
+//   fa_bwd_dkdv_kernel one CTA per (head, 128 keys): K_j, V_j stay in shared
+//                      memory while 128-query blocks of Q, dO stream through
+//                      a ring; S^T = K Q^T and dP^T = V dO^T land in tensor
+//                      memory (keys on the lanes), the compute warps turn
+//                      them into 16-bit P^T and dS^T in place, and
+//                      dV += P^T dO, dK += dS^T Q accumulate in tensor memory.
+//   fa_bwd_dq_kernel   one CTA per (head, 128 queries): S = Q K^T and
+//                      dP = dO V^T per 128-key block, dS in place, dQ += dS K.
+//                      Computing dQ in its own pass (recomputing S and dP
+//                      once more) avoids fp32 atomics on dQ.
+//
+// Warps 0-3: compute (thread = row of the 128-row tile); warp 4: TMA
+// producer; warp 5: tensor-memory allocation and the MMA-issuing thread.
+// Tensor memory (dK/dV kernel): S^T [0,128), dP^T [128,256), dV [256,256+d),
+// dK [256+d,256+2d); (dQ kernel): S [0,128), dP [128,256), dQ [256,256+d).
+// Every wait is bounded as in the forward kernel.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <type_traits>
+
+#include "ptx.cuh"
+
+namespace fa {
+
+enum : int { kBwdElemBF16 = 0, kBwdElemF16 = 1 };
+
+struct BwdArgs {
+  const void* o;         // [BH, N, D]   (D pre-pass)
+  const void* dout;      // [BH, N, D]   (D pre-pass)
+  const float* lse;      // [BH, N] natural log, from the forward
+  float* delta;          // [BH, N] D = rowsum(dO * O)
+  void* dq;              // [BH, N, D]
+  void* dk;              // [BH, N, D]
+  void* dv;              // [BH, N, D]
+  unsigned int* status;  // device status word
+  int BH, N, causal;
+  int nblk;              // ceil(N / 128)
+  float scale;           // softmax scale
+  float scale_log2;      // softmax scale * log2(e)
+  uint64_t wait_limit_ns;
+};
+
+enum : unsigned { kStatusBwd = 16u };
+
+template <int D, int ELEM>
+struct BwdCfg {
+  static constexpr int ROW = D * 2;                          // bytes per 16-bit row
+  static constexpr int SW = ROW >= 128 ? 128 : ROW;          // swizzle span
+  static_assert(SW == 128 || SW == 64, "unsupported head dimension");
+  static constexpr int TILE = 128 * ROW;                      // one 128-row tile
+  static constexpr int FIXED = 2 * TILE;                      // the two resident tiles
+  static constexpr int STAGE = 2 * TILE;                      // the two streamed tiles
+  static constexpr int NS_FIT = (200 * 1024 - FIXED) / STAGE;
+  static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
+  static_assert(NS >= 2, "ring too shallow");
+  static constexpr int BYTES = FIXED + NS * STAGE;
+  static constexpr int NUM_BARS = 2 * NS + 5;
+  static constexpr int SMEM_NEED = 1024 + BYTES + 8 * NUM_BARS;
+  static constexpr int SMEM_BYTES = SMEM_NEED > 120 * 1024 ? SMEM_NEED : 120 * 1024;  // one CTA per SM
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget exceeded");
+  static constexpr int K_STEPS = ROW / 32;                    // 16 elements per MMA K step
+  static constexpr uint32_t FMT = ELEM == 1 ? 0u : 1u;        // f16 : bf16
+  static constexpr uint32_t IDESC_SS = instr_desc(FMT, FMT, 0u, 128, 128);
+  static constexpr uint32_t IDESC_TS = instr_desc(FMT, FMT, 1u, 128, D);
+  static constexpr uint32_t SWZ = SW == 128 ? 2u : 4u;
+  static constexpr uint32_t COL_A = 0, COL_B = 128, COL_ACC0 = 256, COL_ACC1 = 256 + D;
+};
+
+// Barrier slots: fixed tiles loaded, fixed tiles released, ring full/empty,
+// scores ready, P/dS ready, accumulators final.
+template <int NS>
+struct BwdBars {
+  uint32_t base;
+  __device__ __forceinline__ uint32_t fixed_full() const { return base; }
+  __device__ __forceinline__ uint32_t full(int s) const { return base + 8u * (1 + s); }
+  __device__ __forceinline__ uint32_t empty(int s) const { return base + 8u * (1 + NS + s); }
+  __device__ __forceinline__ uint32_t s_full() const { return base + 8u * (1 + 2 * NS); }
+  __device__ __forceinline__ uint32_t p_full() const { return base + 8u * (2 + 2 * NS); }
+  __device__ __forceinline__ uint32_t acc_full() const { return base + 8u * (3 + 2 * NS); }
+  __device__ __forceinline__ uint32_t mma_done() const { return base + 8u * (4 + 2 * NS); }
+};
+
+// ---------------------------------------------------------------- D pre-pass
+// One warp per row: D[r] = sum_c dO[r, c] * O[r, c] in fp32.
+template <int D, int ELEM>
+__global__ void __launch_bounds__(256) bwd_d_kernel(const BwdArgs a) {
+  using T = typename std::conditional<ELEM == 1, __half, __nv_bfloat16>::type;
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= static_cast<long long>(a.BH) * a.N) return;
+  const T* o = reinterpret_cast<const T*>(a.o) + row * D;
+  const T* g = reinterpret_cast<const T*>(a.dout) + row * D;
+  float acc = 0.f;
+#pragma unroll
+  for (int c = lane; c < D; c += 32) {
+    float oc, gc;
+    if constexpr (ELEM == 1) {
+      oc = __half2float(o[c]);
+      gc = __half2float(g[c]);
+    } else {
+      oc = __bfloat162float(o[c]);
+      gc = __bfloat162float(g[c]);
+    }
+    acc = fmaf(oc, gc, acc);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) a.delta[row] = acc;
+}
+
+// ---------------------------------------------------------------- helpers
+template <int D, int ELEM>
+__device__ __forceinline__ void bwd_load_tile(uint32_t dst, const CUtensorMap* map, uint32_t bar, int row0, int bh) {
+  using C = BwdCfg<D, ELEM>;
+#pragma unroll
+  for (int c = 0; c < C::ROW / C::SW; ++c)
+    tma_load_3d(dst + c * 128 * C::SW, map, bar, c * (C::SW / 2), row0, bh);
+}
+
+// A x B^T with both operands K-major 128-row tiles in shared memory.
+template <int D, int ELEM>
+__device__ __forceinline__ void bwd_mma_ss(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
+  using C = BwdCfg<D, ELEM>;
+  const uint64_t da = smem_desc(a_smem, 16, 8 * C::SW, C::SWZ);
+  const uint64_t db = smem_desc(b_smem, 16, 8 * C::SW, C::SWZ);
+#pragma unroll
+  for (int kk = 0; kk < C::K_STEPS; ++kk) {
+    const uint32_t off = ((kk * 32) / C::SW) * (128 * C::SW) + ((kk * 32) % C::SW);
+    mma_f16_ss(d_tmem, da + (off >> 4), db + (off >> 4), C::IDESC_SS, kk > 0);
+  }
+}
+
+// acc (+)= A B with A (128 x 128, 16-bit) in tensor memory at a_tmem and B a
+// 128-row tile in shared memory read N-major (its rows are the K index).
+template <int D, int ELEM>
+__device__ __forceinline__ void bwd_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, bool accumulate) {
+  using C = BwdCfg<D, ELEM>;
+  const uint64_t db = smem_desc(b_smem, 128 * C::SW, 8 * C::SW, C::SWZ);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    mma_f16_ts(d_tmem, a_tmem + kk * 8, db + ((kk * 16 * C::SW) >> 4), C::IDESC_TS, (accumulate || kk > 0) ? 1u : 0u);
+}
+
+template <int ELEM>
+__device__ __forceinline__ uint32_t pack16(float lo, float hi) {
+  return ELEM == 1 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
+}
+
+// Scores of one 32-column chunk turned into 16-bit P and dS (both written
+// back over the first half of their own regions).  Column e of the chunk is
+// the other side's row (query for dK/dV, key for dQ); `valid(e)` masks it.
+struct ChunkIn {
+  uint32_t s[32];
+  uint32_t dp[32];
+};
+
+// 128-row accumulator rows (NC fp32 columns) -> 16-bit global rows, scaled.
+template <int D, int ELEM>
+__device__ __forceinline__ void bwd_store_acc(uint32_t t_acc, void* out, int bh, int N, int row, float mult) {
+  using T = typename std::conditional<ELEM == 1, __half, __nv_bfloat16>::type;
+  T* dst_row = reinterpret_cast<T*>(out) + (static_cast<size_t>(bh) * N + row) * D;
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(t_acc + c * 32, r);
+    tmem_ld_wait(r);
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      pk[e] = pack16<ELEM>(__uint_as_float(r[2 * e]) * mult, __uint_as_float(r[2 * e + 1]) * mult);
+    if (row < N) {
+      uint4* d4 = reinterpret_cast<uint4*>(dst_row + c * 32);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) d4[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- dK, dV
+template <int D, int ELEM>
+__global__ void __launch_bounds__(192, 1)
+    fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                       const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
+                       const BwdArgs a) {
+  using C = BwdCfg<D, ELEM>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint32_t tmem_holder;
+  __shared__ int abort_storage;
+  volatile int* abort_flag = &abort_storage;
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sK = (raw + 1023u) & ~1023u;
+  const uint32_t sV = sK + C::TILE;
+  const uint32_t sRing = sK + C::FIXED;  // stage s: Q at +s*STAGE, dO at +s*STAGE+TILE
+  const BwdBars<C::NS> b{sK + C::BYTES};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x / a.nblk;
+  const int j = blockIdx.x - bh * a.nblk;  // key block
+  const int i0 = a.causal ? j : 0;         // first query block with unmasked scores
+  const int n_i = a.nblk - i0;
+  const uint64_t limit = a.wait_limit_ns;
+
+  if (threadIdx.x == 0) {
+    abort_storage = 0;
+    mbar_init(b.fixed_full(), 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(b.full(s), 1);
+      mbar_init(b.empty(s), 1);
+    }
+    mbar_init(b.s_full(), 1);
+    mbar_init(b.p_full(), 4);
+    mbar_init(b.acc_full(), 1);
+    mbar_init(b.mma_done(), 1);
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_holder;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(b.fixed_full(), 2 * C::TILE);
+      bwd_load_tile<D, ELEM>(sK, &map_k, b.fixed_full(), 128 * j, bh);
+      bwd_load_tile<D, ELEM>(sV, &map_v, b.fixed_full(), 128 * j, bh);
+      bool ok = true;
+      int issued = 0;
+      for (int t = 0; t < n_i && ok; ++t) {
+        const int s = t % C::NS, r = t / C::NS;
+        if (r > 0 && !wait_bounded(b.empty(s), (r - 1) & 1, abort_flag, limit)) {
+          ok = false;
+          break;
+        }
+        const uint32_t dst = sRing + s * C::STAGE;
+        mbar_arrive_expect_tx(b.full(s), 2 * C::TILE);
+        bwd_load_tile<D, ELEM>(dst, &map_q, b.full(s), 128 * (i0 + t), bh);
+        bwd_load_tile<D, ELEM>(dst + C::TILE, &map_do, b.full(s), 128 * (i0 + t), bh);
+        ++issued;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        atomicOr(a.status, kStatusBwd);
+      }
+      volatile int never = 0;
+      bool drained = wait_bounded(b.fixed_full(), 0, &never, limit);
+      for (int t = issued - 1; t >= 0 && t >= issued - C::NS; --t)
+        drained &= wait_bounded(b.full(t % C::NS), (t / C::NS) & 1, &never, limit);
+      if (!drained) atomicOr(a.status, kStatusBwd);
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      bool ok = wait_bounded(b.fixed_full(), 0, abort_flag, limit);
+      for (int t = 0; t < n_i && ok; ++t) {
+        const int s = t % C::NS;
+        if (!wait_bounded(b.full(s), (t / C::NS) & 1, abort_flag, limit)) {
+          ok = false;
+          break;
+        }
+        const uint32_t sQ = sRing + s * C::STAGE, sDO = sQ + C::TILE;
+        bwd_mma_ss<D, ELEM>(tmem + C::COL_A, sK, sQ);   // S^T = K Q^T
+        bwd_mma_ss<D, ELEM>(tmem + C::COL_B, sV, sDO);  // dP^T = V dO^T
+        tc_commit(b.s_full());
+        if (!wait_bounded(b.p_full(), t & 1, abort_flag, limit)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        bwd_mma_ts<D, ELEM>(tmem + C::COL_ACC0, tmem + C::COL_A, sDO, t > 0);  // dV += P^T dO
+        bwd_mma_ts<D, ELEM>(tmem + C::COL_ACC1, tmem + C::COL_B, sQ, t > 0);   // dK += dS^T Q
+        tc_commit(b.empty(s));
+      }
+      if (ok) tc_commit(b.acc_full());
+      if (!ok) {
+        *abort_flag = 1;
+        atomicOr(a.status, kStatusBwd);
+      }
+      tc_commit(b.mma_done());
+      volatile int never = 0;
+      if (!wait_bounded(b.mma_done(), 0, &never, limit)) atomicOr(a.status, kStatusBwd);
+    }
+  } else {
+    // compute warps: thread = key row
+    const int row = warp * 32 + lane;
+    const int key = 128 * j + row;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::COL_A, tP = tmem + lane_off + C::COL_B;
+    const float* lse_h = a.lse + static_cast<size_t>(bh) * a.N;
+    const float* dlt_h = a.delta + static_cast<size_t>(bh) * a.N;
+    bool ok = true;
+    for (int t = 0; t < n_i && ok; ++t) {
+      const int qb = (i0 + t) * 128;
+      ok = __all_sync(0xffffffffu, wait_bounded(b.s_full(), t & 1, abort_flag, limit));
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        ChunkIn in;
+        tmem_ld32(tS + 32 * c, in.s);
+        tmem_ld32(tP + 32 * c, in.dp);
+        tmem_ld_wait(in.s);
+        reg_tie(in.dp);
+        uint32_t pp[16], pd[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float pv[2], dv[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int qq = qb + 32 * c + e + u;
+            const bool valid = qq < a.N && !(a.causal && qq < key);
+            const float lse2 = valid ? lse_h[qq] * 1.4426950408889634f : 0.f;
+            const float dlt = valid ? dlt_h[qq] : 0.f;
+            const float p = valid ? ex2_approx(fmaf(__uint_as_float(in.s[e + u]), a.scale_log2, -lse2)) : 0.f;
+            pv[u] = p;
+            dv[u] = p * (__uint_as_float(in.dp[e + u]) - dlt);
+          }
+          pp[e >> 1] = pack16<ELEM>(pv[0], pv[1]);
+          pd[e >> 1] = pack16<ELEM>(dv[0], dv[1]);
+        }
+        tmem_st16(tS + 16 * c, pp);
+        tmem_st16(tP + 16 * c, pd);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b.p_full());
+    }
+    if (ok) ok = __all_sync(0xffffffffu, wait_bounded(b.acc_full(), 0, abort_flag, limit));
+    if (ok) {
+      tc_fence_after();
+      bwd_store_acc<D, ELEM>(tmem + lane_off + C::COL_ACC0, a.dv, bh, a.N, key, 1.f);
+      bwd_store_acc<D, ELEM>(tmem + lane_off + C::COL_ACC1, a.dk, bh, a.N, key, a.scale);
+    } else {
+      *abort_flag = 1;
+      atomicOr(a.status, kStatusBwd);
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- dQ
+template <int D, int ELEM>
+__global__ void __launch_bounds__(192, 1)
+    fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
+                     const BwdArgs a) {
+  using C = BwdCfg<D, ELEM>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint32_t tmem_holder;
+  __shared__ int abort_storage;
+  volatile int* abort_flag = &abort_storage;
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sQ = (raw + 1023u) & ~1023u;
+  const uint32_t sDO = sQ + C::TILE;
+  const uint32_t sRing = sQ + C::FIXED;  // stage s: K at +s*STAGE, V at +s*STAGE+TILE
+  const BwdBars<C::NS> b{sQ + C::BYTES};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x / a.nblk;
+  const int i = blockIdx.x - bh * a.nblk;  // query block
+  const int n_j = a.causal ? i + 1 : a.nblk;
+  const uint64_t limit = a.wait_limit_ns;
+
+  if (threadIdx.x == 0) {
+    abort_storage = 0;
+    mbar_init(b.fixed_full(), 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(b.full(s), 1);
+      mbar_init(b.empty(s), 1);
+    }
+    mbar_init(b.s_full(), 1);
+    mbar_init(b.p_full(), 4);
+    mbar_init(b.acc_full(), 1);
+    mbar_init(b.mma_done(), 1);
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_holder;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(b.fixed_full(), 2 * C::TILE);
+      bwd_load_tile<D, ELEM>(sQ, &map_q, b.fixed_full(), 128 * i, bh);
+      bwd_load_tile<D, ELEM>(sDO, &map_do, b.fixed_full(), 128 * i, bh);
+      bool ok = true;
+      int issued = 0;
+      for (int t = 0; t < n_j && ok; ++t) {
+        const int s = t % C::NS, r = t / C::NS;
+        if (r > 0 && !wait_bounded(b.empty(s), (r - 1) & 1, abort_flag, limit)) {
+          ok = false;
+          break;
+        }
+        const uint32_t dst = sRing + s * C::STAGE;
+        mbar_arrive_expect_tx(b.full(s), 2 * C::TILE);
+        bwd_load_tile<D, ELEM>(dst, &map_k, b.full(s), 128 * t, bh);
+        bwd_load_tile<D, ELEM>(dst + C::TILE, &map_v, b.full(s), 128 * t, bh);
+        ++issued;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        atomicOr(a.status, kStatusBwd);
+      }
+      volatile int never = 0;
+      bool drained = wait_bounded(b.fixed_full(), 0, &never, limit);
+      for (int t = issued - 1; t >= 0 && t >= issued - C::NS; --t)
+        drained &= wait_bounded(b.full(t % C::NS), (t / C::NS) & 1, &never, limit);
+      if (!drained) atomicOr(a.status, kStatusBwd);
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      bool ok = wait_bounded(b.fixed_full(), 0, abort_flag, limit);
+      for (int t = 0; t < n_j && ok; ++t) {
+        const int s = t % C::NS;
+        if (!wait_bounded(b.full(s), (t / C::NS) & 1, abort_flag, limit)) {
+          ok = false;
+          break;
+        }
+        const uint32_t sK = sRing + s * C::STAGE, sV = sK + C::TILE;
+        bwd_mma_ss<D, ELEM>(tmem + C::COL_A, sQ, sK);   // S = Q K^T
+        bwd_mma_ss<D, ELEM>(tmem + C::COL_B, sDO, sV);  // dP = dO V^T
+        tc_commit(b.s_full());
+        if (!wait_bounded(b.p_full(), t & 1, abort_flag, limit)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        bwd_mma_ts<D, ELEM>(tmem + C::COL_ACC0, tmem + C::COL_A, sK, t > 0);  // dQ += dS K
+        tc_commit(b.empty(s));
+      }
+      if (ok) tc_commit(b.acc_full());
+      if (!ok) {
+        *abort_flag = 1;
+        atomicOr(a.status, kStatusBwd);
+      }
+      tc_commit(b.mma_done());
+      volatile int never = 0;
+      if (!wait_bounded(b.mma_done(), 0, &never, limit)) atomicOr(a.status, kStatusBwd);
+    }
+  } else {
+    // compute warps: thread = query row
+    const int row = warp * 32 + lane;
+    const int qrow = 128 * i + row;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::COL_A, tP = tmem + lane_off + C::COL_B;
+    const bool row_ok = qrow < a.N;
+    const float lse2 = row_ok ? a.lse[static_cast<size_t>(bh) * a.N + qrow] * 1.4426950408889634f : 0.f;
+    const float dlt = row_ok ? a.delta[static_cast<size_t>(bh) * a.N + qrow] : 0.f;
+    bool ok = true;
+    for (int t = 0; t < n_j && ok; ++t) {
+      ok = __all_sync(0xffffffffu, wait_bounded(b.s_full(), t & 1, abort_flag, limit));
+      if (!ok) break;
+      tc_fence_after();
+      const int kb = 128 * t;
+      // keys past the sequence end, or after the query when causal, are masked
+      const int limit_key = (a.causal && qrow < a.N - 1) ? qrow : a.N - 1;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        ChunkIn in;
+        tmem_ld32(tS + 32 * c, in.s);
+        tmem_ld32(tP + 32 * c, in.dp);
+        tmem_ld_wait(in.s);
+        reg_tie(in.dp);
+        uint32_t pd[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float dv[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const bool valid = row_ok && kb + 32 * c + e + u <= limit_key;
+            const float p = valid ? ex2_approx(fmaf(__uint_as_float(in.s[e + u]), a.scale_log2, -lse2)) : 0.f;
+            dv[u] = p * (__uint_as_float(in.dp[e + u]) - dlt);
+          }
+          pd[e >> 1] = pack16<ELEM>(dv[0], dv[1]);
+        }
+        tmem_st16(tS + 16 * c, pd);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b.p_full());
+    }
+    if (ok) ok = __all_sync(0xffffffffu, wait_bounded(b.acc_full(), 0, abort_flag, limit));
+    if (ok) {
+      tc_fence_after();
+      bwd_store_acc<D, ELEM>(tmem + lane_off + C::COL_ACC0, a.dq, bh, a.N, qrow, a.scale);
+    } else {
+      *abort_flag = 1;
+      atomicOr(a.status, kStatusBwd);
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fa

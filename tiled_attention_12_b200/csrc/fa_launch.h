@@ -10,6 +10,7 @@
 namespace fa {
 
 struct FwdArgs;
+struct BwdArgs;
 
 struct FwdLaunch {
   CUtensorMap map_q, map_k, map_v;
@@ -25,5 +26,13 @@ cudaError_t launch_fwd_e4m3(int d, const FwdLaunch& l);
 cudaError_t launch_quantize_e4m3(const void* x, void* x8, float* scales, int BH, int N, int d,
                                  cudaStream_t stream);
 int fwd_smem_bytes(int d, int elem);
+
+struct BwdLaunch {
+  CUtensorMap map_q, map_k, map_v, map_do;
+  const BwdArgs* args;
+  cudaStream_t stream;
+};
+// D pre-pass, dK/dV kernel and dQ kernel, in that order on l.stream.
+cudaError_t launch_bwd(int d, int elem, const BwdLaunch& l);
 
 }  // namespace fa
