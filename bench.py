@@ -300,6 +300,33 @@ def run_ours(args, rank, world, local_rank):
                     del q, k, v, o, lse
                 except Exception as e:  # report, never hide
                     suite[c.name] = {"error": str(e)[:200]}
+        # backward (fa_bwd) on the d=128 shapes: algorithmic FLOPs 2.5x the
+        # forward's (five N x N x d products: S, dP, dV, dK, dQ)
+        for c in list(WORKLOADS["target_d128_noncausal"].cases[:1]) + list(WORKLOADS["b4h16n8192d128_causal"].cases):
+            name = "bwd_" + c.name
+            try:
+                q, k, v = device_inputs(c, salt=2)
+                g = torch.randn(q.shape, device=dev, generator=torch.Generator(device=dev).manual_seed(7)).to(q.dtype)
+                o, lse = fa.fa_fwd(q, k, v, causal=c.causal, softmax_scale=c.softmax_scale)
+                dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+                kw = dict(dq=dq, dk=dk, dv=dv, causal=c.causal, softmax_scale=c.softmax_scale)
+                for _ in range(3):
+                    fa.fa_bwd(q, k, v, o, lse, g, **kw)
+                times = []
+                for _ in range(5):
+                    flush.zero_()
+                    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a0.record(stream)
+                    fa.fa_bwd(q, k, v, o, lse, g, **kw)
+                    a1.record(stream)
+                    torch.cuda.synchronize()
+                    times.append(a0.elapsed_time(a1))
+                ms = statistics.median(times)
+                suite[name] = {"ms": round(ms, 4), "tflops": round(2.5 * c.flops / ms / 1e9, 1),
+                               "note": "backward; FLOPs counted as 2.5x forward"}
+                del q, k, v, g, o, lse, dq, dk, dv
+            except Exception as e:  # report, never hide
+                suite[name] = {"error": str(e)[:200]}
         torch.cuda.synchronize()
         if fa.fa_last_device_status() != 0:
             raise SystemExit("device status reports a timed-out wait in the suite")

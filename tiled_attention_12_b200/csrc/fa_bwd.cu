@@ -21,9 +21,9 @@ cudaError_t launch_bwd_t(const BwdLaunch& l) {
     return e;
   if ((e = cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)) != cudaSuccess)
     return e;
-  kdkdv<<<grid, 192, C::SMEM_BYTES, l.stream>>>(l.map_q, l.map_k, l.map_v, l.map_do, a);
+  kdkdv<<<grid, 320, C::SMEM_BYTES, l.stream>>>(l.map_q, l.map_k, l.map_v, l.map_do, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  kdq<<<grid, 192, C::SMEM_BYTES, l.stream>>>(l.map_q, l.map_k, l.map_v, l.map_do, a);
+  kdq<<<grid, 320, C::SMEM_BYTES, l.stream>>>(l.map_q, l.map_k, l.map_v, l.map_do, a);
   return cudaGetLastError();
 }
 

@@ -20,8 +20,10 @@
 //                      Computing dQ in its own pass (recomputing S and dP
 //                      once more) avoids fp32 atomics on dQ.
 //
-// Warps 0-3: compute (thread = row of the 128-row tile); warp 4: TMA
-// producer; warp 5: tensor-memory allocation and the MMA-issuing thread.
+// Warps 0-7: compute (warp w: rows 32(w%4)..+31 of the 128-row tile, columns
+// 64(w/4)..+63 of the 128x128 score block; two warps per scheduler partition
+// keep the exp2 unit busy); warp 8: TMA producer; warp 9: tensor-memory
+// allocation and the MMA-issuing thread.
 // Tensor memory (dK/dV kernel): S^T [0,128), dP^T [128,256), dV [256,256+d),
 // dK [256+d,256+2d); (dQ kernel): S [0,128), dP [128,256), dQ [256,256+d).
 // Every wait is bounded as in the forward kernel.
@@ -151,8 +153,12 @@ __device__ __forceinline__ void bwd_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uin
   using C = BwdCfg<D, ELEM>;
   const uint64_t db = smem_desc(b_smem, 128 * C::SW, 8 * C::SW, C::SWZ);
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk)
-    mma_f16_ts(d_tmem, a_tmem + kk * 8, db + ((kk * 16 * C::SW) >> 4), C::IDESC_TS, (accumulate || kk > 0) ? 1u : 0u);
+  for (int kk = 0; kk < 8; ++kk) {
+    // packed 16-bit operand: rows 0..63 of K at columns 0..31, rows 64..127 at
+    // columns 64..95 (each compute warp packs inside its own 64-column half)
+    const uint32_t a_col = kk * 8 + (kk >= 4 ? 32u : 0u);
+    mma_f16_ts(d_tmem, a_tmem + a_col, db + ((kk * 16 * C::SW) >> 4), C::IDESC_TS, (accumulate || kk > 0) ? 1u : 0u);
+  }
 }
 
 template <int ELEM>
@@ -192,7 +198,7 @@ __device__ __forceinline__ void bwd_store_acc(uint32_t t_acc, void* out, int bh,
 
 // ---------------------------------------------------------------- dK, dV
 template <int D, int ELEM>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                        const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
                        const BwdArgs a) {
@@ -221,12 +227,12 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(b.empty(s), 1);
     }
     mbar_init(b.s_full(), 1);
-    mbar_init(b.p_full(), 4);
+    mbar_init(b.p_full(), 8);
     mbar_init(b.acc_full(), 1);
     mbar_init(b.mma_done(), 1);
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(&tmem_holder, 512);
     tmem_relinquish();
   }
@@ -235,7 +241,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_holder;
 
-  if (warp == 4) {
+  if (warp == 8) {
     if (lane == 0) {
       mbar_arrive_expect_tx(b.fixed_full(), 2 * C::TILE);
       bwd_load_tile<D, ELEM>(sK, &map_k, b.fixed_full(), 128 * j, bh);
@@ -264,7 +270,7 @@ __global__ void __launch_bounds__(192, 1)
         drained &= wait_bounded(b.full(t % C::NS), (t / C::NS) & 1, &never, limit);
       if (!drained) atomicOr(a.status, kStatusBwd);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     if (lane == 0) {
       bool ok = wait_bounded(b.fixed_full(), 0, abort_flag, limit);
       for (int t = 0; t < n_i && ok; ++t) {
@@ -296,10 +302,11 @@ __global__ void __launch_bounds__(192, 1)
       if (!wait_bounded(b.mma_done(), 0, &never, limit)) atomicOr(a.status, kStatusBwd);
     }
   } else {
-    // compute warps: thread = key row
-    const int row = warp * 32 + lane;
+    // compute warps: thread = key row; warp w covers query columns 64(w/4)..+63
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = quarter * 32 + lane;
     const int key = 128 * j + row;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::COL_A, tP = tmem + lane_off + C::COL_B;
     const float* lse_h = a.lse + static_cast<size_t>(bh) * a.N;
     const float* dlt_h = a.delta + static_cast<size_t>(bh) * a.N;
@@ -310,10 +317,28 @@ __global__ void __launch_bounds__(192, 1)
       if (!ok) break;
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 2 * half; c < 2 * half + 2; ++c) {
         ChunkIn in;
         tmem_ld32(tS + 32 * c, in.s);
         tmem_ld32(tP + 32 * c, in.dp);
+        // LSE and D of the chunk's 32 queries (the same for every lane)
+        const int q0 = qb + 32 * c;
+        float lse2[32], dlt[32];
+        if (q0 + 32 <= a.N && ((reinterpret_cast<uintptr_t>(lse_h + q0) | reinterpret_cast<uintptr_t>(dlt_h + q0)) & 15) == 0) {
+#pragma unroll
+          for (int v4 = 0; v4 < 8; ++v4) {
+            const float4 l4 = reinterpret_cast<const float4*>(lse_h + q0)[v4];
+            const float4 d4 = reinterpret_cast<const float4*>(dlt_h + q0)[v4];
+            lse2[4 * v4] = l4.x; lse2[4 * v4 + 1] = l4.y; lse2[4 * v4 + 2] = l4.z; lse2[4 * v4 + 3] = l4.w;
+            dlt[4 * v4] = d4.x; dlt[4 * v4 + 1] = d4.y; dlt[4 * v4 + 2] = d4.z; dlt[4 * v4 + 3] = d4.w;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            lse2[e] = q0 + e < a.N ? lse_h[q0 + e] : 0.f;
+            dlt[e] = q0 + e < a.N ? dlt_h[q0 + e] : 0.f;
+          }
+        }
         tmem_ld_wait(in.s);
         reg_tie(in.dp);
         uint32_t pp[16], pd[16];
@@ -322,19 +347,17 @@ __global__ void __launch_bounds__(192, 1)
           float pv[2], dv[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const int qq = qb + 32 * c + e + u;
+            const int qq = q0 + e + u;
             const bool valid = qq < a.N && !(a.causal && qq < key);
-            const float lse2 = valid ? lse_h[qq] * 1.4426950408889634f : 0.f;
-            const float dlt = valid ? dlt_h[qq] : 0.f;
-            const float p = valid ? ex2_approx(fmaf(__uint_as_float(in.s[e + u]), a.scale_log2, -lse2)) : 0.f;
-            pv[u] = p;
-            dv[u] = p * (__uint_as_float(in.dp[e + u]) - dlt);
+            const float p = ex2_approx(fmaf(__uint_as_float(in.s[e + u]), a.scale_log2, -lse2[e + u] * 1.4426950408889634f));
+            pv[u] = valid ? p : 0.f;
+            dv[u] = pv[u] * (__uint_as_float(in.dp[e + u]) - dlt[e + u]);
           }
           pp[e >> 1] = pack16<ELEM>(pv[0], pv[1]);
           pd[e >> 1] = pack16<ELEM>(dv[0], dv[1]);
         }
-        tmem_st16(tS + 16 * c, pp);
-        tmem_st16(tP + 16 * c, pd);
+        tmem_st16(tS + 64 * half + 16 * (c - 2 * half), pp);
+        tmem_st16(tP + 64 * half + 16 * (c - 2 * half), pd);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -344,8 +367,11 @@ __global__ void __launch_bounds__(192, 1)
     if (ok) ok = __all_sync(0xffffffffu, wait_bounded(b.acc_full(), 0, abort_flag, limit));
     if (ok) {
       tc_fence_after();
-      bwd_store_acc<D, ELEM>(tmem + lane_off + C::COL_ACC0, a.dv, bh, a.N, key, 1.f);
-      bwd_store_acc<D, ELEM>(tmem + lane_off + C::COL_ACC1, a.dk, bh, a.N, key, a.scale);
+      // warp half 0 stores dV, half 1 stores dK (this thread's key row)
+      if (half == 0)
+        bwd_store_acc<D, ELEM>(tmem + lane_off + C::COL_ACC0, a.dv, bh, a.N, key, 1.f);
+      else
+        bwd_store_acc<D, ELEM>(tmem + lane_off + C::COL_ACC1, a.dk, bh, a.N, key, a.scale);
     } else {
       *abort_flag = 1;
       atomicOr(a.status, kStatusBwd);
@@ -353,7 +379,7 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_before();
   }
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -361,7 +387,7 @@ __global__ void __launch_bounds__(192, 1)
 
 // ---------------------------------------------------------------- dQ
 template <int D, int ELEM>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                      const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
                      const BwdArgs a) {
@@ -389,12 +415,12 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(b.empty(s), 1);
     }
     mbar_init(b.s_full(), 1);
-    mbar_init(b.p_full(), 4);
+    mbar_init(b.p_full(), 8);
     mbar_init(b.acc_full(), 1);
     mbar_init(b.mma_done(), 1);
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(&tmem_holder, 512);
     tmem_relinquish();
   }
@@ -403,7 +429,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_holder;
 
-  if (warp == 4) {
+  if (warp == 8) {
     if (lane == 0) {
       mbar_arrive_expect_tx(b.fixed_full(), 2 * C::TILE);
       bwd_load_tile<D, ELEM>(sQ, &map_q, b.fixed_full(), 128 * i, bh);
@@ -432,7 +458,7 @@ __global__ void __launch_bounds__(192, 1)
         drained &= wait_bounded(b.full(t % C::NS), (t / C::NS) & 1, &never, limit);
       if (!drained) atomicOr(a.status, kStatusBwd);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     if (lane == 0) {
       bool ok = wait_bounded(b.fixed_full(), 0, abort_flag, limit);
       for (int t = 0; t < n_j && ok; ++t) {
@@ -463,10 +489,11 @@ __global__ void __launch_bounds__(192, 1)
       if (!wait_bounded(b.mma_done(), 0, &never, limit)) atomicOr(a.status, kStatusBwd);
     }
   } else {
-    // compute warps: thread = query row
-    const int row = warp * 32 + lane;
+    // compute warps: thread = query row; warp w covers key columns 64(w/4)..+63
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = quarter * 32 + lane;
     const int qrow = 128 * i + row;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::COL_A, tP = tmem + lane_off + C::COL_B;
     const bool row_ok = qrow < a.N;
     const float lse2 = row_ok ? a.lse[static_cast<size_t>(bh) * a.N + qrow] * 1.4426950408889634f : 0.f;
@@ -480,7 +507,7 @@ __global__ void __launch_bounds__(192, 1)
       // keys past the sequence end, or after the query when causal, are masked
       const int limit_key = (a.causal && qrow < a.N - 1) ? qrow : a.N - 1;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 2 * half; c < 2 * half + 2; ++c) {
         ChunkIn in;
         tmem_ld32(tS + 32 * c, in.s);
         tmem_ld32(tP + 32 * c, in.dp);
@@ -493,12 +520,12 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const bool valid = row_ok && kb + 32 * c + e + u <= limit_key;
-            const float p = valid ? ex2_approx(fmaf(__uint_as_float(in.s[e + u]), a.scale_log2, -lse2)) : 0.f;
-            dv[u] = p * (__uint_as_float(in.dp[e + u]) - dlt);
+            const float p = ex2_approx(fmaf(__uint_as_float(in.s[e + u]), a.scale_log2, -lse2));
+            dv[u] = valid ? p * (__uint_as_float(in.dp[e + u]) - dlt) : 0.f;
           }
           pd[e >> 1] = pack16<ELEM>(dv[0], dv[1]);
         }
-        tmem_st16(tS + 16 * c, pd);
+        tmem_st16(tS + 64 * half + 16 * (c - 2 * half), pd);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -508,7 +535,7 @@ __global__ void __launch_bounds__(192, 1)
     if (ok) ok = __all_sync(0xffffffffu, wait_bounded(b.acc_full(), 0, abort_flag, limit));
     if (ok) {
       tc_fence_after();
-      bwd_store_acc<D, ELEM>(tmem + lane_off + C::COL_ACC0, a.dq, bh, a.N, qrow, a.scale);
+      if (half == 0) bwd_store_acc<D, ELEM>(tmem + lane_off + C::COL_ACC0, a.dq, bh, a.N, qrow, a.scale);
     } else {
       *abort_flag = 1;
       atomicOr(a.status, kStatusBwd);
@@ -516,7 +543,7 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_before();
   }
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
