@@ -13,8 +13,12 @@ from __future__ import annotations
 import math
 
 
-def brute_attention(q, k, v, scale: float, causal: bool):
-    """q, k, v: nested lists [N][d] of floats.  Returns (o [N][dv], lse [N])."""
+def brute_attention(q, k, v, scale: float, causal: bool, keep=None):
+    """q, k, v: nested lists [N][d] of floats.  Returns (o [N][dv], lse [N]).
+
+    ``keep(i, j)``, when given, further restricts which keys query i sees
+    (block-sparse attention); a query that sees no key gets a zero row and
+    LSE = -inf (an empty softmax)."""
     n_q, n_k = len(q), len(k)
     d = len(q[0])
     dv = len(v[0])
@@ -24,10 +28,16 @@ def brute_attention(q, k, v, scale: float, causal: bool):
         for j in range(n_k):
             if causal and j > i:
                 continue
+            if keep is not None and not keep(i, j):
+                continue
             dot = 0.0
             for c in range(d):
                 dot += q[i][c] * k[j][c]
             scores.append((j, dot * scale))
+        if not scores:
+            o.append([0.0] * dv)
+            lse.append(-math.inf)
+            continue
         big = max(s for _, s in scores)
         weights = [(j, math.exp(s - big)) for j, s in scores]
         total = sum(w for _, w in weights)
