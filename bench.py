@@ -137,12 +137,25 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- our arm
+def block_sparse_pair_count(mask, N: int, causal: bool, block: int = 128) -> float:
+    """Kept (query, key) pairs of a block mask: block sizes product, with the
+    diagonal blocks' lower triangle (diagonal included) when causal."""
+    import torch
+
+    nb = mask.shape[-1]
+    sizes = torch.clamp(N - torch.arange(nb, dtype=torch.float64) * block, max=block)
+    pairs = sizes[:, None] * sizes[None, :]
+    if causal:
+        pairs = torch.tril(pairs, diagonal=-1) + torch.diag(sizes * (sizes + 1) / 2)
+    return float((mask.double().cpu() * pairs).sum())
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
 
     import tiled_attention_12_b200 as fa
     from tiled_attention_12_b200.dist import aggregate_throughput, max_over_ranks
-    from tiled_attention_12_b200.synth import WORKLOADS
+    from tiled_attention_12_b200.synth import WORKLOADS, make_block_mask
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -325,6 +338,38 @@ def run_ours(args, rank, world, local_rank):
                 suite[name] = {"ms": round(ms, 4), "tflops": round(2.5 * c.flops / ms / 1e9, 1),
                                "note": "backward; FLOPs counted as 2.5x forward"}
                 del q, k, v, g, o, lse, dq, dk, dv
+            except Exception as e:  # report, never hide
+                suite[name] = {"error": str(e)[:200]}
+        # block-sparse forward (fa_fwd_block_sparse): B4 H16 N8192 d128 with a
+        # sliding window of +-3 key blocks plus key block 0, and a random half
+        # of the blocks; FLOPs = 4 d per kept (query, key) pair
+        bc = WORKLOADS["target_d128_noncausal"].cases[0]
+        for label, kind, causal in (("window3", "window", False), ("window3_causal", "window", True),
+                                    ("random50", "random", False)):
+            name = f"bs_{label}_" + bc.name.replace("_noncausal", "")
+            try:
+                q, k, v = device_inputs(bc, salt=3)
+                mask = make_block_mask(bc.B, bc.H, bc.N, kind, 0.5, window=3, seed=1).to(dev)
+                o = torch.empty_like(v)
+                lse = torch.empty((bc.B, bc.H, bc.N), device=dev, dtype=torch.float32)
+                kw = dict(o=o, lse=lse, causal=causal, softmax_scale=bc.softmax_scale)
+                for _ in range(3):
+                    fa.fa_fwd_block_sparse(q, k, v, mask, **kw)
+                times = []
+                for _ in range(5):
+                    flush.zero_()
+                    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a0.record(stream)
+                    fa.fa_fwd_block_sparse(q, k, v, mask, **kw)
+                    a1.record(stream)
+                    torch.cuda.synchronize()
+                    times.append(a0.elapsed_time(a1))
+                ms = statistics.median(times)
+                flops = block_sparse_pair_count(mask, bc.N, causal) * 4.0 * bc.d
+                suite[name] = {"ms": round(ms, 4), "tflops": round(flops / ms / 1e9, 1),
+                               "density": round(float(mask.float().mean()), 3),
+                               "note": "block-sparse; includes the plan pre-pass"}
+                del q, k, v, o, lse, mask
             except Exception as e:  # report, never hide
                 suite[name] = {"error": str(e)[:200]}
         torch.cuda.synchronize()

@@ -103,6 +103,28 @@ fa_status fa_fwd_fp8(const void* q8, const float* q_scale, const void* k8, const
                      float softmax_scale, int causal, void* stream);
 
 /*
+ * fa_fwd_block_sparse — fa_fwd restricted to chosen 128 x 128 blocks of the
+ * attention matrix ("深度解析注意力机制的变体与演进", Block Sparse Attention:
+ * the matrix is cut into fixed-size blocks and only some are computed, full
+ * attention inside a computed block, none through a skipped one).
+ *   block_mask : device pointer, uint8 [B, H, ceil(N/128), ceil(N/128)],
+ *                row-major; entry (b, h, i, j) nonzero = query rows
+ *                [128 i, 128 i + 128) attend to keys [128 j, 128 j + 128).
+ *                With causal = 1 the causal mask applies on top (blocks above
+ *                the diagonal are never computed, whatever the mask says).
+ *   Other arguments, layouts and dtypes as in fa_fwd.
+ * A query row with no computed key gets a zero output row and LSE = -inf.
+ * Ceiling: ceil(N/128) <= 512 (N <= 65536); larger N -> FA_ERR_UNSUPPORTED.
+ * The library builds a per-call plan (the K/V tiles each 256-row work tile
+ * visits) in a workspace grown on demand with cudaMalloc and freed by
+ * fa_release; the mask is read on `stream` before the attention kernel and
+ * may be reused or freed once that work is done.
+ */
+fa_status fa_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                              int B, int H, int N, int d, float softmax_scale, int causal,
+                              const uint8_t* block_mask, fa_dtype dtype, void* stream);
+
+/*
  * fa_bwd — gradients of fa_fwd by recomputation ("从理论到实现…" §2.2: no
  * intermediate is stored; S and P are recomputed from Q, K and the forward's
  * LSE).  With P = exp(softmax_scale * Q K^T - LSE) (causal mask as in fa_fwd):

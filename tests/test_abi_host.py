@@ -62,3 +62,23 @@ def test_other_entry_points_reject_bad_arguments():
     assert L.fa_fwd_fp8(P, P, P, P, P, P * 2, None, 1, 1, 16, 64, 0.1, 0, None) == B.FA_ERR_UNSUPPORTED
     assert L.fa_fwd_fp8(P, None, P, P, P, P * 2, None, 1, 1, 16, 128, 0.1, 0, None) == B.FA_ERR_INVALID
     assert L.fa_fwd_fp8(P, P + 1, P, P, P, P * 2, None, 1, 1, 16, 128, 0.1, 0, None) == B.FA_ERR_INVALID
+
+
+def test_block_sparse_rejects_bad_arguments_without_cuda():
+    L = B.load()
+    f = L.fa_fwd_block_sparse
+    assert f(P, P, P, P * 2, None, 1, 1, 256, 64, 0.1, 0, None, 0, None) == B.FA_ERR_INVALID        # null mask
+    assert f(P, P, P, P * 2, None, 1, 1, 65537, 64, 0.1, 0, P, 0, None) == B.FA_ERR_UNSUPPORTED     # > 512 tiles
+    assert f(P, P, P, P * 2, None, 1, 1, 256, 48, 0.1, 0, P, 0, None) == B.FA_ERR_UNSUPPORTED       # d = 48
+    assert f(P, P, P, P * 2, None, 1, 1, 256, 64, 0.1, 0, P, 2, None) == B.FA_ERR_UNSUPPORTED       # e4m3, d = 64
+    assert f(P, P, P, P, None, 1, 1, 256, 64, 0.1, 0, P, 0, None) == B.FA_ERR_INVALID               # o aliases q
+    assert f(P, P, P, P * 2, None, 1, 1, 256, 64, 0.1, 3, P, 0, None) == B.FA_ERR_INVALID           # causal = 3
+
+
+def test_block_mask_generator_is_seeded_and_shaped():
+    from tiled_attention_12_b200.synth import make_block_mask
+    a = make_block_mask(2, 3, 1000, "random", 0.4, seed=5)
+    assert a.shape == (2, 3, 8, 8) and a.dtype.is_floating_point is False
+    assert (a == make_block_mask(2, 3, 1000, "random", 0.4, seed=5)).all()
+    w = make_block_mask(1, 1, 1024, "window", window=1)
+    assert w[0, 0, 5].tolist() == [1, 0, 0, 0, 1, 1, 1, 0]

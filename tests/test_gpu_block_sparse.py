@@ -1,0 +1,123 @@
+"""GPU parity of the block-sparse forward (fa_fwd_block_sparse) against the
+fp64 block-sparse oracle ("深度解析注意力机制的变体与演进", Block Sparse
+Attention), and bit-identity with the dense forward when every block is kept."""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import tiled_attention_12_b200 as fa
+from oracle import dequantize_e4m3_tiles, quantize_e4m3_tiles
+from oracle.block_sparse import attention_block_sparse_ref, attention_block_sparse_rows
+from parity_util import TOL_16, gate, sample_rows
+from tiled_attention_12_b200.synth import Case, make_block_mask, make_qkv
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _check(o, lse, ro, rl, dtype, what):
+    """Rows the mask empties: exactly zero and LSE = -inf.  Others: the 16-bit gate."""
+    o = o.float().cpu().double().numpy()
+    lse = lse.double().cpu().numpy()
+    empty = np.isneginf(rl)
+    assert np.array_equal(np.isneginf(lse), empty), what
+    assert np.all(o[empty] == 0.0), what
+    live = ~empty
+    if live.any():
+        gate(o[live], ro[live], lse[live], rl[live], tol=TOL_16, out_dtype=dtype, what=what)
+
+
+def _run(case, mask, dtype=torch.bfloat16, code=None):
+    q, k, v = make_qkv(case, dtype=dtype)
+    o, lse = fa.fa_fwd_block_sparse(q.to(DEV), k.to(DEV), v.to(DEV), mask.to(DEV), causal=case.causal, dtype=code)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status() == 0
+    return q, k, v, o, lse
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [200, 1000])
+@pytest.mark.parametrize("d", [32, 64, 128])
+def test_all_blocks_is_bit_identical_to_dense(d, N, causal, dtype):
+    case = Case("bs_ones", 2, 3, N, d, causal, seed=N + d)
+    mask = make_block_mask(2, 3, N, "ones")
+    q, k, v, o, lse = _run(case, mask, dtype)
+    od, ld = fa.fa_fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=causal)
+    torch.cuda.synchronize()
+    assert torch.equal(o, od) and torch.equal(lse, ld)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("density", [0.3, 0.7])
+@pytest.mark.parametrize("N", [300, 777, 1280])
+@pytest.mark.parametrize("d", [32, 64, 128])
+def test_random_masks_against_oracle(d, N, density, causal):
+    case = Case("bs_rand", 1, 3, N, d, causal, seed=7 * N + d)
+    mask = make_block_mask(1, 3, N, "random", density, seed=N + int(10 * density))
+    mask[0, 1, 1, :] = 0          # query rows 128..255 of head 1 keep nothing
+    mask[0, 2, :, 0] = 1          # head 2: every row keeps key block 0
+    q, k, v, o, lse = _run(case, mask)
+    ro, rl = attention_block_sparse_ref(q, k, v, case.softmax_scale, causal, mask)
+    _check(o, lse, ro, rl, torch.bfloat16, f"d{d} N{N} p{density} c{causal}")
+
+
+@pytest.mark.parametrize("d", [32, 128])
+def test_no_blocks_gives_zero_rows_and_minus_inf(d):
+    case = Case("bs_zero", 1, 2, 500, d, False, seed=3)
+    q, k, v, o, lse = _run(case, make_block_mask(1, 2, 500, "zeros"))
+    assert torch.count_nonzero(o).item() == 0
+    assert bool(torch.isneginf(lse).all())
+
+
+def test_causal_diagonal_removed_empties_first_rows():
+    """Causal with block (0, 0) removed: rows 0..127 see no key at all."""
+    case = Case("bs_diag", 1, 1, 384, 64, True, seed=4)
+    mask = make_block_mask(1, 1, 384, "ones")
+    mask[0, 0, 0, 0] = 0
+    q, k, v, o, lse = _run(case, mask)
+    ro, rl = attention_block_sparse_ref(q, k, v, case.softmax_scale, True, mask)
+    assert np.all(np.isneginf(rl[0, 0, :128])) and np.all(np.isfinite(rl[0, 0, 128:]))
+    _check(o, lse, ro, rl, torch.bfloat16, "diag removed")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d,kind", [(128, "window"), (64, "random"), (32, "window")])
+def test_many_work_tiles_sampled_rows(d, kind, causal):
+    """More work tiles than SMs (each CTA walks several plans through the
+    two-slot feed); checked on sampled rows of a few heads."""
+    B, H, N = 2, 8, 8192
+    case = Case("bs_big", B, H, N, d, causal, seed=11 + d)
+    mask = make_block_mask(B, H, N, kind, 0.25, window=3, seed=d)
+    q, k, v, o, lse = _run(case, mask)
+    rows = sample_rows(N, seed=d, n_random=64)
+    for b, h in ((0, 0), (1, 5), (1, 7)):
+        ro, rl = attention_block_sparse_rows(q, k, v, case.softmax_scale, causal, mask, b, h, rows)
+        _check(o[b, h][torch.as_tensor(rows, device=DEV)], lse[b, h][torch.as_tensor(rows, device=DEV)],
+               ro, rl, torch.bfloat16, f"{kind} d{d} ({b},{h})")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_e4m3_against_dequantised_oracle(causal):
+    """FA_E4M3 dtype: Q and K quantised per 128-row tile by the library; the
+    oracle is fed the dequantised codes (the FP8 reading of the dense tests)."""
+    case = Case("bs_fp8", 1, 2, 640, 128, causal, seed=21)
+    mask = make_block_mask(1, 2, 640, "random", 0.5, seed=2)
+    q, k, v, o, lse = _run(case, mask, code=fa.FA_E4M3)
+    cq, sq = quantize_e4m3_tiles(q)
+    ck, sk = quantize_e4m3_tiles(k)
+    ro, rl = attention_block_sparse_ref(dequantize_e4m3_tiles(cq, sq), dequantize_e4m3_tiles(ck, sk), v,
+                                        case.softmax_scale, causal, mask)
+    _check(o, lse, ro, rl, torch.bfloat16, "e4m3")
+
+
+def test_e4m3_all_blocks_is_bit_identical_to_dense():
+    case = Case("bs_fp8_ones", 1, 2, 900, 128, True, seed=22)
+    mask = make_block_mask(1, 2, 900, "ones")
+    q, k, v, o, lse = _run(case, mask, code=fa.FA_E4M3)
+    od, ld = fa.fa_fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=True, dtype=fa.FA_E4M3)
+    torch.cuda.synchronize()
+    assert torch.equal(o, od) and torch.equal(lse, ld)

@@ -48,14 +48,15 @@ def load():
     L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     L.fa_fwd_e4m3_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
+    L.fa_fwd_block_sparse.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, i, vp]
     L.fa_last_device_status.argtypes = [vp]
     L.fa_status_string.argtypes = [i]
     L.fa_status_string.restype = ctypes.c_char_p
     L.fa_release.argtypes = []
     L.fa_debug_set_wait_limit.argtypes = [ctypes.c_uint64]
     L.fa_debug_withhold_arrival.argtypes = [i]
-    for name in ("fa_fwd", "fa_bwd", "fa_quantize_e4m3", "fa_fwd_fp8", "fa_fwd_e4m3_noalloc", "fa_last_device_status",
-                 "fa_release",
+    for name in ("fa_fwd", "fa_bwd", "fa_fwd_block_sparse", "fa_quantize_e4m3", "fa_fwd_fp8",
+                 "fa_fwd_e4m3_noalloc", "fa_last_device_status", "fa_release",
                  "fa_debug_set_wait_limit", "fa_debug_withhold_arrival"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
@@ -115,6 +116,34 @@ def fa_fwd(q, k, v, o=None, lse=None, softmax_scale=None, causal=False, dtype=No
     st = load().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, scale,
                        int(bool(causal)), code, _stream(stream))
     _check(st, "fa_fwd")
+    return o, lse
+
+
+def fa_fwd_block_sparse(q, k, v, block_mask, o=None, lse=None, softmax_scale=None, causal=False, dtype=None,
+                        stream=None, want_lse=True):
+    """Block-sparse forward: block_mask is a uint8 CUDA tensor
+    [B, H, ceil(N/128), ceil(N/128)] (nonzero = computed block).  Returns (o, lse)."""
+    import torch
+
+    for t in (q, k, v):
+        if not (t.is_cuda and t.is_contiguous() and t.dim() == 4):
+            raise ValueError("q, k, v must be contiguous 4-D CUDA tensors")
+    if q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v shapes differ")
+    B, H, N, d = q.shape
+    nb = (N + 127) // 128
+    if not (block_mask.is_cuda and block_mask.is_contiguous() and block_mask.dtype == torch.uint8
+            and tuple(block_mask.shape) == (B, H, nb, nb)):
+        raise ValueError(f"block_mask must be a contiguous uint8 CUDA tensor of shape {(B, H, nb, nb)}")
+    code = _dtype_code(q) if dtype is None else dtype
+    if o is None:
+        o = torch.empty_like(v)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
+    scale = (1.0 / d ** 0.5) if softmax_scale is None else float(softmax_scale)
+    st = load().fa_fwd_block_sparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, scale,
+                                    int(bool(causal)), _ptr(block_mask), code, _stream(stream))
+    _check(st, "fa_fwd_block_sparse")
     return o, lse
 
 

@@ -42,7 +42,20 @@ struct DeviceState {
   size_t ws_bytes = 0;
   float* bwd_ws = nullptr;         // backward: D = rowsum(dO * O)
   size_t bwd_ws_bytes = 0;
+  void* plan_ws = nullptr;         // block-sparse plan rows
+  size_t plan_ws_bytes = 0;
 };
+
+// Grows a per-device workspace to at least `need` bytes (under g_mu).
+fa_status grow(void** ptr, size_t* bytes, size_t need) {
+  if (*bytes >= need) return FA_OK;
+  if (*ptr) cudaFree(*ptr);
+  *ptr = nullptr;
+  *bytes = 0;
+  if (cudaMalloc(ptr, need) != cudaSuccess) return FA_ERR_CUDA;
+  *bytes = need;
+  return FA_OK;
+}
 
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
@@ -128,7 +141,7 @@ int group_heads(int BH, int N, int d, int qk_bytes) {
 
 fa_status launch_attention(DeviceState* ds, int elem, const void* q, const void* k, const void* v, void* o,
                            float* lse, const float* q_scale, const float* k_scale, int BH, int N, int d,
-                           float softmax_scale, int causal, cudaStream_t stream) {
+                           float softmax_scale, int causal, cudaStream_t stream, const uint16_t* plan = nullptr) {
   fa::FwdLaunch l;
   const int qk_bytes = elem == fa::kElemE4M3 ? 1 : 2;
   fa_status st;
@@ -159,6 +172,11 @@ fa_status launch_attention(DeviceState* ds, int elem, const void* q, const void*
   }
   l.grid = a.n_work < ds->sms ? a.n_work : ds->sms;
   a.group_heads = group_heads(BH, N, d, qk_bytes);
+  if (plan != nullptr) {
+    a.plan = plan;
+    a.plan_stride = fa::block_sparse_plan_stride(N);
+    a.plan_row_bytes = 2 * (fa::kPlanHeader + 3 * a.plan_stride);
+  }
   l.args = &a;
   l.stream = stream;
   cudaError_t e;
@@ -169,6 +187,34 @@ fa_status launch_attention(DeviceState* ds, int elem, const void* q, const void*
   else
     e = fa::launch_fwd_e4m3(d, l);
   return map_cuda(e);
+}
+
+// e4m3 codes and per-tile scales of q and k in the library workspace.
+struct Quantised {
+  uint8_t* q8;
+  uint8_t* k8;
+  float* qs;
+  float* ks;
+};
+
+fa_status quantise_qk(DeviceState* ds, const void* q, const void* k, int BH, int N, int d, cudaStream_t s,
+                      Quantised* out) {
+  const size_t elems = static_cast<size_t>(BH) * N * d;
+  const size_t n_scales = static_cast<size_t>(BH) * ((N + 127) / 128);
+  const size_t codes_bytes = (elems + 255) & ~static_cast<size_t>(255);
+  const size_t need = 2 * codes_bytes + 2 * n_scales * sizeof(float);
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    fa_status st = grow(&ds->ws, &ds->ws_bytes, need);
+    if (st != FA_OK) return st;
+  }
+  out->q8 = static_cast<uint8_t*>(ds->ws);
+  out->k8 = out->q8 + codes_bytes;
+  out->qs = reinterpret_cast<float*>(out->k8 + codes_bytes);
+  out->ks = out->qs + n_scales;
+  if (fa::launch_quantize_e4m3(q, out->q8, out->qs, BH, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (fa::launch_quantize_e4m3(k, out->k8, out->ks, BH, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
+  return FA_OK;
 }
 
 }  // namespace
@@ -197,27 +243,47 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                                                 softmax_scale, causal, s);
 
   // FA_E4M3: quantise q and k into the library workspace, then attend.
-  const size_t elems = static_cast<size_t>(BH) * N * d;
-  const size_t n_scales = static_cast<size_t>(BH) * ((N + 127) / 128);
-  const size_t codes_bytes = (elems + 255) & ~static_cast<size_t>(255);
-  const size_t need = 2 * codes_bytes + 2 * n_scales * sizeof(float);
+  Quantised qz;
+  if ((st = quantise_qk(ds, q, k, BH, N, d, s, &qz)) != FA_OK) return st;
+  return launch_attention(ds, fa::kElemE4M3, qz.q8, qz.k8, v, o, lse, qz.qs, qz.ks, BH, N, d, softmax_scale, causal,
+                          s);
+}
+
+fa_status fa_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+                              int d, float softmax_scale, int causal, const uint8_t* block_mask, fa_dtype dtype,
+                              void* stream) {
+  if (dtype != FA_BF16 && dtype != FA_FP16 && dtype != FA_E4M3) return FA_ERR_INVALID;
+  fa_status st = check_shape(B, H, N, d);
+  if (st != FA_OK) return st;
+  if (dtype == FA_E4M3 && d != 128) return FA_ERR_UNSUPPORTED;
+  if ((N + 127) / 128 > fa::kPlanMaxTiles) return FA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o || !block_mask) return FA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)))
+    return FA_ERR_INVALID;
+  if (!scale_ok(softmax_scale) || (causal != 0 && causal != 1)) return FA_ERR_INVALID;
+  if (o == q || o == k || o == v) return FA_ERR_INVALID;
+
+  DeviceState* ds = nullptr;
+  if ((st = device_state(&ds)) != FA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  uint16_t* plan = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    if (ds->ws_bytes < need) {
-      if (ds->ws) cudaFree(ds->ws);
-      ds->ws = nullptr;
-      ds->ws_bytes = 0;
-      if (cudaMalloc(&ds->ws, need) != cudaSuccess) return FA_ERR_CUDA;
-      ds->ws_bytes = need;
-    }
+    if ((st = grow(&ds->plan_ws, &ds->plan_ws_bytes, fa::block_sparse_plan_bytes(BH, N))) != FA_OK) return st;
+    plan = static_cast<uint16_t*>(ds->plan_ws);
   }
-  uint8_t* q8 = static_cast<uint8_t*>(ds->ws);
-  uint8_t* k8 = q8 + codes_bytes;
-  float* qs = reinterpret_cast<float*>(k8 + codes_bytes);
-  float* ks = qs + n_scales;
-  if (fa::launch_quantize_e4m3(q, q8, qs, BH, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
-  if (fa::launch_quantize_e4m3(k, k8, ks, BH, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
-  return launch_attention(ds, fa::kElemE4M3, q8, k8, v, o, lse, qs, ks, BH, N, d, softmax_scale, causal, s);
+  if (fa::launch_block_sparse_plan(block_mask, plan, BH, N, causal, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (dtype == FA_BF16)
+    return launch_attention(ds, fa::kElemBF16, q, k, v, o, lse, nullptr, nullptr, BH, N, d, softmax_scale, causal, s,
+                            plan);
+  if (dtype == FA_FP16)
+    return launch_attention(ds, fa::kElemF16, q, k, v, o, lse, nullptr, nullptr, BH, N, d, softmax_scale, causal, s,
+                            plan);
+  Quantised qz;
+  if ((st = quantise_qk(ds, q, k, BH, N, d, s, &qz)) != FA_OK) return st;
+  return launch_attention(ds, fa::kElemE4M3, qz.q8, qz.k8, v, o, lse, qz.qs, qz.ks, BH, N, d, softmax_scale, causal,
+                          s, plan);
 }
 
 fa_status fa_quantize_e4m3(const void* x, void* x8, float* scales, int B, int H, int N, int d, void* stream) {
@@ -341,6 +407,7 @@ fa_status fa_release(void) {
   DeviceState& s = g_dev[dev];
   if (s.ws) cudaFree(s.ws);
   if (s.bwd_ws) cudaFree(s.bwd_ws);
+  if (s.plan_ws) cudaFree(s.plan_ws);
   if (s.status) cudaFree(s.status);
   s.ready = false;
   s.sms = 0;
@@ -350,6 +417,8 @@ fa_status fa_release(void) {
   s.ws_bytes = 0;
   s.bwd_ws = nullptr;
   s.bwd_ws_bytes = 0;
+  s.plan_ws = nullptr;
+  s.plan_ws_bytes = 0;
   return FA_OK;
 }
 

@@ -4,19 +4,21 @@
 namespace fa {
 
 cudaError_t launch_fwd_bf16(int d, const FwdLaunch& l) {
+  if (l.args->plan != nullptr) return launch_fwd_sparse(d, kElemBF16, l);
   switch (d) {
-    case 32: return launch_fwd_t<32, kElemBF16>(l);
-    case 64: return launch_fwd_t<64, kElemBF16>(l);
-    case 128: return launch_fwd_t<128, kElemBF16>(l);
+    case 32: return launch_fwd_t<32, kElemBF16, false>(l);
+    case 64: return launch_fwd_t<64, kElemBF16, false>(l);
+    case 128: return launch_fwd_t<128, kElemBF16, false>(l);
     default: return cudaErrorInvalidValue;
   }
 }
 
 cudaError_t launch_fwd_f16(int d, const FwdLaunch& l) {
+  if (l.args->plan != nullptr) return launch_fwd_sparse(d, kElemF16, l);
   switch (d) {
-    case 32: return launch_fwd_t<32, kElemF16>(l);
-    case 64: return launch_fwd_t<64, kElemF16>(l);
-    case 128: return launch_fwd_t<128, kElemF16>(l);
+    case 32: return launch_fwd_t<32, kElemF16, false>(l);
+    case 64: return launch_fwd_t<64, kElemF16, false>(l);
+    case 128: return launch_fwd_t<128, kElemF16, false>(l);
     default: return cudaErrorInvalidValue;
   }
 }

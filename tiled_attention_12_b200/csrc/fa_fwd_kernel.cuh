@@ -30,6 +30,14 @@
 // order, so S_i(j+1) may overwrite P_i(j) after PV_i(j) is issued, and the
 // completion of S_i(j+1) also tells its warpgroup that PV_i(j) is finished
 // (the O rescale for step j+1 needs that).
+//
+// Block-sparse mode ("深度解析注意力机制的变体与演进", Block Sparse Attention:
+// only chosen blocks of the attention matrix are computed): a plan built
+// from a per-head 128 x 128 block mask lists, per work tile, the K/V tiles
+// either Q tile needs (the union, loaded once) and each Q tile's own list.
+// The TMA thread copies the work tile's plan into shared memory with the
+// tile index; every role walks it instead of the dense prefix 0..n-1, and a
+// Q tile with no computed block writes zero rows and LSE = -inf.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -58,6 +66,17 @@ enum : int { kElemBF16 = 0, kElemF16 = 1, kElemE4M3 = 2 };
 // Status bits written to the device status word when a wait gives up.
 enum : unsigned { kStatusProducer = 1u, kStatusMma = 2u, kStatusSoftmax = 4u, kStatusDrain = 8u };
 
+// Block-sparse plan row of one work tile (uint16 entries):
+//   [0] union count  [1] Q tile 0 count  [2] Q tile 1 count  [3..7] zero
+//   [8 .. 8+stride)          union: (kv tile << 2) | used by tile 0 | used by tile 1 << 1
+//   [8+stride .. 8+2stride)  Q tile 0's kv tiles in order
+//   [8+2stride .. 8+3stride) Q tile 1's kv tiles in order
+// stride = ceil(kv tiles / 8) * 8, so a row is a whole number of 16 bytes.
+constexpr int kPlanHeader = 8;
+constexpr int kPlanMaxTiles = 512;  // kv tiles per head: N <= 65536
+constexpr int kPlanSlotBytes = 2 * (kPlanHeader + 3 * kPlanMaxTiles);
+static_assert(kPlanSlotBytes % 16 == 0, "plan slots must be whole 16-byte units");
+
 struct FwdArgs {
   void* o;                 // [BH, N, D], element type of V
   float* lse;              // [BH, N] fp32 or nullptr
@@ -75,6 +94,9 @@ struct FwdArgs {
   int n_qtiles;            // ceil(N / 128): scale entries per head
   float scale_log2;        // softmax_scale * log2(e)
   uint64_t wait_limit_ns;  // bound for every in-kernel wait
+  const uint16_t* plan;    // block-sparse plan rows [n_work][plan_row] or nullptr (dense)
+  int plan_stride;         // entries per list in a plan row
+  int plan_row_bytes;      // bytes per plan row (2 * (8 + 3 * plan_stride))
 };
 
 template <int D, int ELEM>
@@ -99,7 +121,8 @@ struct FwdCfg {
   static constexpr int NUM_BARS = 21 + 2 * NS;
   // at least 120 KB so that two CTAs never share an SM (each holds all 512
   // tensor-memory columns; a second resident CTA would only wait)
-  static constexpr int SMEM_NEED = 1024 + TILE_BYTES + 8 * NUM_BARS;
+  static constexpr int PLAN_OFFSET = (TILE_BYTES + 8 * NUM_BARS + 127) / 128 * 128;  // from sQ
+  static constexpr int SMEM_NEED = 1024 + PLAN_OFFSET + 2 * kPlanSlotBytes;
   static constexpr int SMEM_BYTES = SMEM_NEED > 120 * 1024 ? SMEM_NEED : 120 * 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget exceeded");
   static constexpr int K_STEPS_QK = QK_ROW / 32;   // 32 bytes of K per S MMA (16 x 16-bit or 32 x 8-bit)
@@ -217,20 +240,28 @@ __device__ __forceinline__ void record_failure(const FwdArgs& a, volatile int* a
 // counter, so each CTA picks up the next tile as soon as it is free.  The
 // TMA thread fetches the index and publishes it in a 2-slot shared-memory
 // ring; the MMA issuer(s) and the eight softmax warps each take it from
-// there and release the slot.  -1 ends the loop.
+// there and release the slot.  -1 ends the loop.  In block-sparse mode the
+// slot also carries the work tile's plan row (a bulk copy counted on the
+// same barrier), and consumers release the slot only when they are done
+// with the work tile.
 struct TileFeed {
   uint32_t full0, empty0;     // barrier addresses of slot 0 (slot 1 follows at +8)
   volatile int* ring;         // [2]
+  const uint16_t* plan0;      // plan slot 0 (slot 1 follows at + kPlanSlotBytes)
+  uint32_t plan0_addr;        // shared-memory address of plan slot 0
+  bool defer;                 // block-sparse: release after the work tile
 };
 
-template <int NS>
-__device__ __forceinline__ TileFeed make_feed(const Bars<NS>& b, volatile int* ring) {
-  return TileFeed{b.feed_full(0), b.feed_empty(0), ring};
+template <bool BS, int NS>
+__device__ __forceinline__ TileFeed make_feed(const Bars<NS>& b, volatile int* ring, uint32_t plan_addr,
+                                              const uint16_t* plan_ptr) {
+  return TileFeed{b.feed_full(0), b.feed_empty(0), ring, plan_ptr, plan_addr, BS};
 }
 
-__device__ __forceinline__ int feed_produce(const FwdArgs& a, const TileFeed& f, int& k, volatile int* abort_flag,
-                                            uint64_t limit, bool& ok) {
-  const int slot = k & 1;
+template <bool BS>
+__device__ __forceinline__ int feed_produce(const FwdArgs& a, const TileFeed& f, int& k, int& slot,
+                                            volatile int* abort_flag, uint64_t limit, bool& ok) {
+  slot = k & 1;
   if (k >= 2 && !wait_bounded(f.empty0 + 8u * slot, ((k >> 1) - 1) & 1, abort_flag, limit)) {
     ok = false;
     return -1;
@@ -238,30 +269,45 @@ __device__ __forceinline__ int feed_produce(const FwdArgs& a, const TileFeed& f,
   int w = static_cast<int>(atomicAdd(a.sched, 1u));
   if (w >= a.n_work) w = -1;
   f.ring[slot] = w;
-  mbar_arrive(f.full0 + 8u * slot);
+  if (BS && w >= 0) {
+    const WorkTile t = decode_work(a, w);
+    const size_t row = static_cast<size_t>(t.bh) * a.n_qpairs + t.tp;
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(a.plan) + row * a.plan_row_bytes;
+    mbar_arrive_expect_tx(f.full0 + 8u * slot, a.plan_row_bytes);
+    bulk_load(f.plan0_addr + slot * kPlanSlotBytes, src, a.plan_row_bytes, f.full0 + 8u * slot);
+  } else {
+    mbar_arrive(f.full0 + 8u * slot);
+  }
   ++k;
   return w;
 }
 
 // Single-thread consumer (an MMA issuer).
-__device__ __forceinline__ int feed_take(const TileFeed& f, int& k, volatile int* abort_flag, uint64_t limit,
-                                         bool& ok) {
-  const int slot = k & 1;
+template <bool BS>
+__device__ __forceinline__ int feed_take(const TileFeed& f, int& k, int& slot, volatile int* abort_flag,
+                                         uint64_t limit, bool& ok) {
+  slot = k & 1;
   if (!wait_bounded(f.full0 + 8u * slot, (k >> 1) & 1, abort_flag, limit)) {
     ok = false;
     return -1;
   }
   const int w = f.ring[slot];
-  mbar_arrive(f.empty0 + 8u * slot);
+  if (!BS || w < 0) mbar_arrive(f.empty0 + 8u * slot);
   ++k;
   return w;
 }
 
+template <bool BS>
+__device__ __forceinline__ void feed_release(const TileFeed& f, int slot) {
+  if (BS) mbar_arrive(f.empty0 + 8u * slot);
+}
+
 // Whole-warp consumer (a softmax warp): every lane gets the index, lane 0
 // releases the slot.
-__device__ __forceinline__ int feed_take_warp(const TileFeed& f, int& k, int lane, volatile int* abort_flag,
-                                              uint64_t limit, bool& ok) {
-  const int slot = k & 1;
+template <bool BS>
+__device__ __forceinline__ int feed_take_warp(const TileFeed& f, int& k, int& slot, int lane,
+                                              volatile int* abort_flag, uint64_t limit, bool& ok) {
+  slot = k & 1;
   const bool got = __all_sync(0xffffffffu, wait_bounded(f.full0 + 8u * slot, (k >> 1) & 1, abort_flag, limit));
   if (!got) {
     ok = false;
@@ -269,16 +315,67 @@ __device__ __forceinline__ int feed_take_warp(const TileFeed& f, int& k, int lan
   }
   const int w = f.ring[slot];
   __syncwarp();
-  if (lane == 0) mbar_arrive(f.empty0 + 8u * slot);
+  if (lane == 0 && (!BS || w < 0)) mbar_arrive(f.empty0 + 8u * slot);
   ++k;
   return w;
+}
+
+template <bool BS>
+__device__ __forceinline__ void feed_release_warp(const TileFeed& f, int slot, int lane) {
+  if constexpr (BS) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(f.empty0 + 8u * slot);
+  }
+}
+
+// The K/V tiles of one work tile.  Dense: Q tile i uses tiles 0..n_i-1 and
+// the pair loads 0..max(n_0, n_1)-1.  Block-sparse: the lists of the plan row
+// in shared memory.
+struct Plan {
+  int nkv;                      // K/V tiles loaded for the work tile
+  int n0, n1;                   // K/V tiles each Q tile uses
+  const uint16_t* uni;          // union entries, or nullptr when dense
+  const uint16_t *own0, *own1;  // each Q tile's kv tiles
+};
+
+template <bool BS>
+__device__ __forceinline__ Plan make_plan(const FwdArgs& a, const WorkTile& t, const TileFeed& f, int slot) {
+  Plan p;
+  if constexpr (!BS) {
+    const int q0 = t.tp * 256;
+    p.n0 = kv_tiles(a, q0);
+    p.n1 = kv_tiles(a, q0 + 128);
+    p.nkv = p.n0 > p.n1 ? p.n0 : p.n1;
+    p.uni = nullptr;
+    p.own0 = p.own1 = nullptr;
+  } else {
+    const uint16_t* row = reinterpret_cast<const uint16_t*>(reinterpret_cast<const uint8_t*>(f.plan0) +
+                                                            slot * kPlanSlotBytes);
+    p.nkv = row[0];
+    p.n0 = row[1];
+    p.n1 = row[2];
+    p.uni = row + kPlanHeader;
+    p.own0 = p.uni + a.plan_stride;
+    p.own1 = p.own0 + a.plan_stride;
+  }
+  return p;
+}
+
+// K/V tile of union entry u; whether Q tile i uses it; Q tile i's s-th tile.
+__device__ __forceinline__ int plan_n(const Plan& p, int i) { return i ? p.n1 : p.n0; }
+__device__ __forceinline__ int plan_tile(const Plan& p, int u) { return p.uni ? (p.uni[u] >> 2) : u; }
+__device__ __forceinline__ bool plan_uses(const Plan& p, int u, int i) {
+  return p.uni ? ((p.uni[u] >> i) & 1) != 0 : u < plan_n(p, i);
+}
+__device__ __forceinline__ int plan_own(const Plan& p, int i, int s) {
+  return p.uni ? (i ? p.own1 : p.own0)[s] : s;
 }
 
 // ---------------------------------------------------------------- producer
 // One thread.  Per work tile: the Q tiles it needs, then K_j, V_j for every
 // K/V step into the ring.  Stage `it % NS` is reused in round `it / NS` once
 // the MMA thread has released round `it / NS - 1`.
-template <int D, int ELEM>
+template <int D, int ELEM, bool BS>
 __device__ __forceinline__ void producer_role(const FwdArgs& a, const Bars<FwdCfg<D, ELEM>::NS> b, uint32_t sQ,
                                               uint32_t sKV, const CUtensorMap* map_q, const CUtensorMap* map_k,
                                               const CUtensorMap* map_v, const TileFeed feed,
@@ -294,11 +391,18 @@ __device__ __forceinline__ void producer_role(const FwdArgs& a, const Bars<FwdCf
   bool ok = true;
   int feed_k = 0;
   while (ok) {
-    const int w = feed_produce(a, feed, feed_k, abort_flag, limit, ok);
+    int slot;
+    const int w = feed_produce<BS>(a, feed, feed_k, slot, abort_flag, limit, ok);
     if (w < 0) break;
     const WorkTile t = decode_work(a, w);
     const int q0 = t.tp * 256;
-    const int n0 = kv_tiles(a, q0), n1 = kv_tiles(a, q0 + 128);
+    // block-sparse: the plan row this thread just copied must have landed
+    if (BS && !wait_bounded(feed.full0 + 8u * slot, ((feed_k - 1) >> 1) & 1, abort_flag, limit)) {
+      ok = false;
+      break;
+    }
+    const Plan p = make_plan<BS>(a, t, feed, slot);
+    const int n0 = p.n0, n1 = p.n1;
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const int n = i ? n1 : n0;
@@ -315,8 +419,8 @@ __device__ __forceinline__ void producer_role(const FwdArgs& a, const Bars<FwdCf
                     q0 + i * 128, t.bh);
       ++use;
     }
-    const int nkv = n0 > n1 ? n0 : n1;
-    for (int j = 0; ok && j < nkv; ++j) {
+    for (int u = 0; ok && u < p.nkv; ++u) {
+      const int j = plan_tile(p, u);
 #pragma unroll
       for (int kind = 0; kind < 2; ++kind) {
         const int s = kv_it % C::NS;
@@ -364,7 +468,7 @@ __device__ __forceinline__ void producer_role(const FwdArgs& a, const Bars<FwdCf
 // One thread issues every tcgen05.mma.  Descriptors are built once per
 // operand base and advanced by adding (byte offset >> 4) to the start-address
 // field, which cannot overflow for shared-memory addresses below 256 KB.
-template <int D, int ELEM>
+template <int D, int ELEM, bool BS>
 __device__ __forceinline__ void mma_role(const FwdArgs& a, const Bars<FwdCfg<D, ELEM>::NS> b, uint32_t sQ_addr,
                                          uint32_t sKV_addr, uint32_t tmem, const TileFeed feed,
                                          volatile int* abort_flag) {
@@ -419,69 +523,148 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const Bars<FwdCfg<D, 
 
   bool ok = true;
   int feed_k = 0;
-  while (ok) {
-    const int w = feed_take(feed, feed_k, abort_flag, limit, ok);
-    if (w < 0) break;
-    const WorkTile t = decode_work(a, w);
-    const int q0 = t.tp * 256;
-    const int n0 = kv_tiles(a, q0), n1 = kv_tiles(a, q0 + 128);
-    const int nkv = n0 > n1 ? n0 : n1;
-    if (n0 > 0 && !wait_bounded(b.q_full(0), (q_use0++) & 1, abort_flag, limit)) { ok = false; break; }
-    if (n1 > 0 && !wait_bounded(b.q_full(1), (q_use1++) & 1, abort_flag, limit)) { ok = false; break; }
-    int sk = kv_it % C::NS;
-    if (!wait_bounded(b.kv_full(sk), (kv_it / C::NS) & 1, abort_flag, limit)) { ok = false; break; }
-    ++kv_it;
-    tc_fence_after();
-    if (n0 > 0) {
-      issue_s(0, sk);
-      tc_commit(b.s_full(0));
-      if (n0 == 1) tc_commit(b.q_empty(0));
-    }
-    if (n1 > 0) {
-      issue_s(1, sk);
-      tc_commit(b.s_full(1));
-      if (n1 == 1) tc_commit(b.q_empty(1));
-    }
-    tc_commit(b.kv_empty(sk));
-    for (int j = 0; j < nkv; ++j) {
-      const int sv = kv_it % C::NS;
-      FA_TRACE_EV(2, 40, j);
-      if (!wait_bounded(b.kv_full(sv), (kv_it / C::NS) & 1, abort_flag, limit)) { ok = false; break; }
-      FA_TRACE_EV(2, 41, j);
+  if constexpr (!BS) {
+    // dense: Q tile i uses K/V tiles 0..n_i-1
+    while (ok) {
+      int slot;
+      const int w = feed_take<BS>(feed, feed_k, slot, abort_flag, limit, ok);
+      if (w < 0) break;
+      const WorkTile t = decode_work(a, w);
+      const int q0 = t.tp * 256;
+      const int n0 = kv_tiles(a, q0), n1 = kv_tiles(a, q0 + 128);
+      const int nkv = n0 > n1 ? n0 : n1;
+      if (n0 > 0 && !wait_bounded(b.q_full(0), (q_use0++) & 1, abort_flag, limit)) { ok = false; break; }
+      if (n1 > 0 && !wait_bounded(b.q_full(1), (q_use1++) & 1, abort_flag, limit)) { ok = false; break; }
+      int sk = kv_it % C::NS;
+      if (!wait_bounded(b.kv_full(sk), (kv_it / C::NS) & 1, abort_flag, limit)) { ok = false; break; }
       ++kv_it;
       tc_fence_after();
-      if (j < n0) {
-        if (!wait_p_and_issue(0, sv, j > 0, p_cnt0)) { ok = false; break; }
-        if (j == n0 - 1) tc_commit(b.o_full(0));
+      if (n0 > 0) {
+        issue_s(0, sk);
+        tc_commit(b.s_full(0));
+        if (n0 == 1) tc_commit(b.q_empty(0));
       }
-      const bool next = j + 1 < nkv;
-      int sk2 = 0;
-      if (next) {
-        sk2 = kv_it % C::NS;
-        FA_TRACE_EV(2, 42, j + 1);
-        if (!wait_bounded(b.kv_full(sk2), (kv_it / C::NS) & 1, abort_flag, limit)) { ok = false; break; }
-        FA_TRACE_EV(2, 43, j + 1);
+      if (n1 > 0) {
+        issue_s(1, sk);
+        tc_commit(b.s_full(1));
+        if (n1 == 1) tc_commit(b.q_empty(1));
+      }
+      tc_commit(b.kv_empty(sk));
+      for (int j = 0; j < nkv; ++j) {
+        const int sv = kv_it % C::NS;
+        FA_TRACE_EV(2, 40, j);
+        if (!wait_bounded(b.kv_full(sv), (kv_it / C::NS) & 1, abort_flag, limit)) { ok = false; break; }
+        FA_TRACE_EV(2, 41, j);
         ++kv_it;
         tc_fence_after();
-        if (j + 1 < n0) {
-          issue_s(0, sk2);
-          tc_commit(b.s_full(0));
-          if (j + 1 == n0 - 1) tc_commit(b.q_empty(0));
+        if (j < n0) {
+          if (!wait_p_and_issue(0, sv, j > 0, p_cnt0)) { ok = false; break; }
+          if (j == n0 - 1) tc_commit(b.o_full(0));
+        }
+        const bool next = j + 1 < nkv;
+        int sk2 = 0;
+        if (next) {
+          sk2 = kv_it % C::NS;
+          FA_TRACE_EV(2, 42, j + 1);
+          if (!wait_bounded(b.kv_full(sk2), (kv_it / C::NS) & 1, abort_flag, limit)) { ok = false; break; }
+          FA_TRACE_EV(2, 43, j + 1);
+          ++kv_it;
+          tc_fence_after();
+          if (j + 1 < n0) {
+            issue_s(0, sk2);
+            tc_commit(b.s_full(0));
+            if (j + 1 == n0 - 1) tc_commit(b.q_empty(0));
+          }
+        }
+        if (j < n1) {
+          if (!wait_p_and_issue(1, sv, j > 0, p_cnt1)) { ok = false; break; }
+          if (j == n1 - 1) tc_commit(b.o_full(1));
+        }
+        tc_commit(b.kv_empty(sv));
+        if (next) {
+          if (j + 1 < n1) {
+            issue_s(1, sk2);
+            tc_commit(b.s_full(1));
+            if (j + 1 == n1 - 1) tc_commit(b.q_empty(1));
+          }
+          tc_commit(b.kv_empty(sk2));
         }
       }
-      if (j < n1) {
-        if (!wait_p_and_issue(1, sv, j > 0, p_cnt1)) { ok = false; break; }
-        if (j == n1 - 1) tc_commit(b.o_full(1));
+    }
+  } else {
+    // block-sparse: walk the plan's union; Q tile i takes the entries marked
+    // for it (the counters replace the dense prefix bounds)
+    while (ok) {
+      int slot;
+      const int w = feed_take<BS>(feed, feed_k, slot, abort_flag, limit, ok);
+      if (w < 0) break;
+      const WorkTile t = decode_work(a, w);
+      const Plan p = make_plan<BS>(a, t, feed, slot);
+      const int n0 = p.n0, n1 = p.n1, nkv = p.nkv;
+      if (nkv == 0) {
+        feed_release<BS>(feed, slot);
+        continue;
       }
-      tc_commit(b.kv_empty(sv));
-      if (next) {
-        if (j + 1 < n1) {
-          issue_s(1, sk2);
-          tc_commit(b.s_full(1));
-          if (j + 1 == n1 - 1) tc_commit(b.q_empty(1));
+      if (n0 > 0 && !wait_bounded(b.q_full(0), (q_use0++) & 1, abort_flag, limit)) { ok = false; break; }
+      if (n1 > 0 && !wait_bounded(b.q_full(1), (q_use1++) & 1, abort_flag, limit)) { ok = false; break; }
+      // per Q tile: S products issued, P V products issued
+      int s0 = 0, s1 = 0, v0 = 0, v1 = 0;
+      int sk = kv_it % C::NS;
+      if (!wait_bounded(b.kv_full(sk), (kv_it / C::NS) & 1, abort_flag, limit)) { ok = false; break; }
+      ++kv_it;
+      tc_fence_after();
+      if (plan_uses(p, 0, 0)) {
+        issue_s(0, sk);
+        tc_commit(b.s_full(0));
+        if (++s0 == n0) tc_commit(b.q_empty(0));
+      }
+      if (plan_uses(p, 0, 1)) {
+        issue_s(1, sk);
+        tc_commit(b.s_full(1));
+        if (++s1 == n1) tc_commit(b.q_empty(1));
+      }
+      tc_commit(b.kv_empty(sk));
+      for (int j = 0; j < nkv; ++j) {
+        const int sv = kv_it % C::NS;
+        FA_TRACE_EV(2, 40, j);
+        if (!wait_bounded(b.kv_full(sv), (kv_it / C::NS) & 1, abort_flag, limit)) { ok = false; break; }
+        FA_TRACE_EV(2, 41, j);
+        ++kv_it;
+        tc_fence_after();
+        if (plan_uses(p, j, 0)) {
+          if (!wait_p_and_issue(0, sv, v0 > 0, p_cnt0)) { ok = false; break; }
+          if (++v0 == n0) tc_commit(b.o_full(0));
         }
-        tc_commit(b.kv_empty(sk2));
+        const bool next = j + 1 < nkv;
+        int sk2 = 0;
+        if (next) {
+          sk2 = kv_it % C::NS;
+          FA_TRACE_EV(2, 42, j + 1);
+          if (!wait_bounded(b.kv_full(sk2), (kv_it / C::NS) & 1, abort_flag, limit)) { ok = false; break; }
+          FA_TRACE_EV(2, 43, j + 1);
+          ++kv_it;
+          tc_fence_after();
+          if (plan_uses(p, j + 1, 0)) {
+            issue_s(0, sk2);
+            tc_commit(b.s_full(0));
+            if (++s0 == n0) tc_commit(b.q_empty(0));
+          }
+        }
+        if (plan_uses(p, j, 1)) {
+          if (!wait_p_and_issue(1, sv, v1 > 0, p_cnt1)) { ok = false; break; }
+          if (++v1 == n1) tc_commit(b.o_full(1));
+        }
+        tc_commit(b.kv_empty(sv));
+        if (next) {
+          if (plan_uses(p, j + 1, 1)) {
+            issue_s(1, sk2);
+            tc_commit(b.s_full(1));
+            if (++s1 == n1) tc_commit(b.q_empty(1));
+          }
+          tc_commit(b.kv_empty(sk2));
+        }
       }
+      feed_release<BS>(feed, slot);
     }
   }
   if (!ok) record_failure(a, abort_flag, kStatusMma);
@@ -650,9 +833,27 @@ __device__ __forceinline__ void epilogue_row(const FwdArgs& a, uint32_t t_o, int
     a.lse[static_cast<size_t>(bh) * a.N + qrow] = (m + __log2f(l)) * 0.69314718055994531f;
 }
 
+// A row that keeps no score (block-sparse, every block of its Q tile skipped):
+// an empty softmax, so a zero output row and LSE = -inf.
+template <int D, int ELEM>
+__device__ __forceinline__ void empty_row(const FwdArgs& a, int bh, int qrow) {
+  if (qrow >= a.N) return;
+  using OutT = typename std::conditional<ELEM == kElemF16, __half, __nv_bfloat16>::type;
+  uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<OutT*>(a.o) + (static_cast<size_t>(bh) * a.N + qrow) * D);
+#pragma unroll
+  for (int v = 0; v < D * 2 / 16; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+  if (a.lse != nullptr) a.lse[static_cast<size_t>(bh) * a.N + qrow] = -INFINITY;
+}
+
+// Keys of K/V tile j that some row of the Q tile starting at q_start must
+// not see: the causal diagonal tile and the tile holding the sequence end.
+__device__ __forceinline__ bool tile_needs_mask(const FwdArgs& a, int j, int q_start) {
+  return (a.causal && j == (q_start >> 7)) || j == ((a.N - 1) >> 7);
+}
+
 // Aliased layout (d = 128): P overwrites the first 64 columns of S, and the
 // MMA warp's order (S_i(j+1) after P_i(j) V) sequences the reuse.
-template <int D, int ELEM>
+template <int D, int ELEM, bool BS>
 __device__ __forceinline__ void softmax_role(const FwdArgs& a, const Bars<FwdCfg<D, ELEM>::NS> b, uint32_t tmem,
                                              int warp, int lane, const TileFeed feed, volatile int* abort_flag) {
   using C = FwdCfg<D, ELEM>;
@@ -677,19 +878,27 @@ __device__ __forceinline__ void softmax_role(const FwdArgs& a, const Bars<FwdCfg
     int feed_k = 0;
     while (true) {
       bool fed = true;
-      const int w = feed_take_warp(feed, feed_k, lane, abort_flag, limit, fed);
+      int slot;
+      const int w = feed_take_warp<BS>(feed, feed_k, slot, lane, abort_flag, limit, fed);
       if (!fed) return false;
       if (w < 0) break;
       const WorkTile t = decode_work(a, w);
+      const Plan p = make_plan<BS>(a, t, feed, slot);
       const int q_start = t.tp * 256 + wg * 128;
-      const int nkv = kv_tiles(a, q_start);
-      if (nkv == 0) continue;
+      const int nkv = plan_n(p, wg);
+      const uint16_t* own = p.uni ? (wg ? p.own1 : p.own0) : nullptr;  // block-sparse: this tile's list
       const int qrow = q_start + row;
+      if (nkv == 0) {
+        feed_release_warp<BS>(feed, slot, lane);
+        empty_row<D, ELEM>(a, t.bh, qrow);
+        continue;
+      }
       float sl2_q = a.scale_log2;
       if constexpr (ELEM == kElemE4M3) sl2_q = a.scale_log2 / a.q_scale[t.bh * a.n_qtiles + (q_start >> 7)];
       float m = -INFINITY;  // running max, log2 units of the scaled score
       float l = 0.f;        // running sum of exponentials
-      for (int j = 0; j < nkv; ++j) {
+      for (int step = 0; step < nkv; ++step) {
+        const int j = own ? own[step] : step;
         if (lane == 0 && wq == 0) FA_TRACE_EV(wg, 0 + 10 * wg, j);
         if (!wait_warp(s_full, s_cnt)) return false;
         ++s_cnt;
@@ -699,10 +908,10 @@ __device__ __forceinline__ void softmax_role(const FwdArgs& a, const Bars<FwdCfg
         if constexpr (ELEM == kElemE4M3) sl2 = sl2_q / a.k_scale[t.bh * a.n_qtiles + j];
         uint32_t sr[4][32];
         load_s_row(t_s, sr);
-        if (j == nkv - 1) mask_row(sr, j * 128, (a.causal && qrow < a.N - 1) ? qrow : a.N - 1);
+        if (BS ? tile_needs_mask(a, j, q_start) : step == nkv - 1) mask_row(sr, j * 128, (a.causal && qrow < a.N - 1) ? qrow : a.N - 1);
         const float mx = row_max(sr) * sl2;
         if (lane == 0 && wq == 0) FA_TRACE_EV(wg, 2 + 10 * wg, j);
-        if (j == 0) {
+        if (step == 0) {
           m = mx;
         } else if (__any_sync(0xffffffffu, mx - m > C::TAU)) {
           const float m_new = fmaxf(m, mx);
@@ -727,6 +936,7 @@ __device__ __forceinline__ void softmax_role(const FwdArgs& a, const Bars<FwdCfg
         }
         l += sum_acc(acc_a, acc_b);
       }
+      feed_release_warp<BS>(feed, slot, lane);
       // epilogue: O / l -> global, LSE
       if (!wait_warp(o_full, o_cnt)) return false;
       ++o_cnt;
@@ -744,7 +954,7 @@ __device__ __forceinline__ void softmax_role(const FwdArgs& a, const Bars<FwdCfg
 // the MMA issuer computes S_i(j+1) while this step's exponentials run, and it
 // writes P_i(j) only once P_i(j-1) V has completed (p_free), which also makes
 // O_i safe to rescale.
-template <int D, int ELEM>
+template <int D, int ELEM, bool BS>
 __device__ __forceinline__ void softmax_role_decoupled(const FwdArgs& a, const Bars<FwdCfg<D, ELEM>::NS> b,
                                                        uint32_t tmem, int warp, int lane, const TileFeed feed,
                                                        volatile int* abort_flag) {
@@ -774,18 +984,26 @@ __device__ __forceinline__ void softmax_role_decoupled(const FwdArgs& a, const B
     int feed_k = 0;
     while (true) {
       bool fed = true;
-      const int w = feed_take_warp(feed, feed_k, lane, abort_flag, limit, fed);
+      int slot;
+      const int w = feed_take_warp<BS>(feed, feed_k, slot, lane, abort_flag, limit, fed);
       if (!fed) return false;
       if (w < 0) break;
       const WorkTile t = decode_work(a, w);
+      const Plan p = make_plan<BS>(a, t, feed, slot);
       const int q_start = t.tp * 256 + wg * 128;
-      const int nkv = kv_tiles(a, q_start);
-      if (nkv == 0) continue;
+      const int nkv = plan_n(p, wg);
+      const uint16_t* own = p.uni ? (wg ? p.own1 : p.own0) : nullptr;  // block-sparse: this tile's list
       const int qrow = q_start + row;
+      if (nkv == 0) {
+        feed_release_warp<BS>(feed, slot, lane);
+        empty_row<D, ELEM>(a, t.bh, qrow);
+        continue;
+      }
       const float sl2 = a.scale_log2;
       float m = -INFINITY;
       float l = 0.f;
-      for (int j = 0; j < nkv; ++j) {
+      for (int step = 0; step < nkv; ++step) {
+        const int j = own ? own[step] : step;
         if (lane == 0 && wq == 0) FA_TRACE_EV(wg, 0 + 10 * wg, j);
         if (!wait_warp(b.s_full(wg), s_cnt)) return false;
         ++s_cnt;
@@ -795,11 +1013,11 @@ __device__ __forceinline__ void softmax_role_decoupled(const FwdArgs& a, const B
         load_s_row(t_s, sr);
         arrive_warp(b.s_free(wg));          // S_i may be overwritten now
         if (lane == 0 && wq == 0) FA_TRACE_EV(wg, 2 + 10 * wg, j);
-        if (j == nkv - 1) mask_row(sr, j * 128, (a.causal && qrow < a.N - 1) ? qrow : a.N - 1);
+        if (BS ? tile_needs_mask(a, j, q_start) : step == nkv - 1) mask_row(sr, j * 128, (a.causal && qrow < a.N - 1) ? qrow : a.N - 1);
         const float mx = row_max(sr) * sl2;
         bool rescale = false;
         float alpha = 1.f;
-        if (j == 0) {
+        if (step == 0) {
           m = mx;
         } else if (__any_sync(0xffffffffu, mx - m > C::TAU)) {
           const float m_new = fmaxf(m, mx);
@@ -829,6 +1047,7 @@ __device__ __forceinline__ void softmax_role_decoupled(const FwdArgs& a, const B
         ++p_writes;
         l += sum_acc(acc_a, acc_b);
       }
+      feed_release_warp<BS>(feed, slot, lane);
       if (!wait_warp(b.o_full(wg), o_cnt)) return false;
       ++o_cnt;
       tc_fence_after();
@@ -848,7 +1067,7 @@ __device__ __forceinline__ void softmax_role_decoupled(const FwdArgs& a, const B
 // counts two arrivals); an issuer whose tile needs fewer K/V tiles (causal)
 // still releases the extra stages, after they are loaded, so the ring's
 // phases advance in step.
-template <int D, int ELEM>
+template <int D, int ELEM, bool BS>
 __device__ __forceinline__ void mma_role_decoupled(const FwdArgs& a, const Bars<FwdCfg<D, ELEM>::NS> b, const int i,
                                                    uint32_t sQ_addr, uint32_t sKV_addr, uint32_t tmem,
                                                    const TileFeed feed, volatile int* abort_flag) {
@@ -902,43 +1121,97 @@ __device__ __forceinline__ void mma_role_decoupled(const FwdArgs& a, const Bars<
 
   bool ok = true;
   int feed_k = 0;
-  while (ok) {
-    const int w = feed_take(feed, feed_k, abort_flag, limit, ok);
-    if (w < 0) break;
-    const WorkTile t = decode_work(a, w);
-    const int q0 = t.tp * 256;
-    const int n0 = kv_tiles(a, q0), n1 = kv_tiles(a, q0 + 128);
-    const int nkv = n0 > n1 ? n0 : n1;
-    const int n = i ? n1 : n0;
-    if (n > 0) {
-      if (!wait_bounded(b.q_full(i), (q_use++) & 1, abort_flag, limit)) { ok = false; break; }
-      int sk = acquire(pos);
-      if (sk < 0 || !issue_s(sk)) { ok = false; break; }
-      if (n == 1) tc_commit(b.q_empty(i));
-      tc_commit(b.kv_empty(sk));
-      for (int j = 0; j < n; ++j) {
-        if (j + 1 < n) {
-          sk = acquire(pos + 2);
-          if (sk < 0 || !issue_s(sk)) { ok = false; break; }
-          if (j + 1 == n - 1) tc_commit(b.q_empty(i));
-          tc_commit(b.kv_empty(sk));
+  if constexpr (!BS) {
+    // dense: this tile uses K/V tiles 0..n-1 of the work tile and releases
+    // the rest
+    while (ok) {
+      int slot;
+      const int w = feed_take<BS>(feed, feed_k, slot, abort_flag, limit, ok);
+      if (w < 0) break;
+      const WorkTile t = decode_work(a, w);
+      const int q0 = t.tp * 256;
+      const int n0 = kv_tiles(a, q0), n1 = kv_tiles(a, q0 + 128);
+      const int nkv = n0 > n1 ? n0 : n1;
+      const int n = i ? n1 : n0;
+      if (n > 0) {
+        if (!wait_bounded(b.q_full(i), (q_use++) & 1, abort_flag, limit)) { ok = false; break; }
+        int sk = acquire(pos);
+        if (sk < 0 || !issue_s(sk)) { ok = false; break; }
+        if (n == 1) tc_commit(b.q_empty(i));
+        tc_commit(b.kv_empty(sk));
+        for (int j = 0; j < n; ++j) {
+          if (j + 1 < n) {
+            sk = acquire(pos + 2);
+            if (sk < 0 || !issue_s(sk)) { ok = false; break; }
+            if (j + 1 == n - 1) tc_commit(b.q_empty(i));
+            tc_commit(b.kv_empty(sk));
+          }
+          const int sv = acquire(pos + 1);
+          if (sv < 0 || !issue_pv(sv, j > 0)) { ok = false; break; }
+          if (j == n - 1) tc_commit(b.o_full(i));
+          tc_commit(b.kv_empty(sv));
+          pos += 2;
         }
-        const int sv = acquire(pos + 1);
-        if (sv < 0 || !issue_pv(sv, j > 0)) { ok = false; break; }
-        if (j == n - 1) tc_commit(b.o_full(i));
-        tc_commit(b.kv_empty(sv));
+        if (!ok) break;
+      }
+      // release-only for the K/V tiles of this work tile that tile i skips
+      for (int j = n; j < nkv && ok; ++j) {
+        for (int kind = 0; kind < 2; ++kind) {
+          const int st = acquire(pos + kind);
+          if (st < 0) { ok = false; break; }
+          mbar_arrive(b.kv_empty(st));
+        }
         pos += 2;
       }
-      if (!ok) break;
     }
-    // release-only for the K/V tiles of this work tile that tile i skips
-    for (int j = n; j < nkv && ok; ++j) {
-      for (int kind = 0; kind < 2; ++kind) {
-        const int st = acquire(pos + kind);
-        if (st < 0) { ok = false; break; }
-        mbar_arrive(b.kv_empty(st));
+  } else {
+    // P_i V for the union entry whose S_i was issued last (ring position pv_pos)
+    auto flush_pv = [&](int pv_pos, int n, int& v) -> bool {
+      const int sv = acquire(pv_pos);
+      if (sv < 0 || !issue_pv(sv, v > 0)) return false;
+      if (++v == n) tc_commit(b.o_full(i));
+      tc_commit(b.kv_empty(sv));
+      return true;
+    };
+    while (ok) {
+      int slot;
+      const int w = feed_take<BS>(feed, feed_k, slot, abort_flag, limit, ok);
+      if (w < 0) break;
+      const WorkTile t = decode_work(a, w);
+      const Plan p = make_plan<BS>(a, t, feed, slot);
+      const int n = plan_n(p, i), nkv = p.nkv;
+      if (n > 0 && !wait_bounded(b.q_full(i), (q_use++) & 1, abort_flag, limit)) { ok = false; break; }
+      // Walk the union in ring order.  Entry u holds ring positions pos + 2u
+      // (K) and pos + 2u + 1 (V).  S_i(u) is issued before P_i V of the
+      // previous used entry when the two are adjacent; across entries this tile
+      // skips, the pending P V goes first and the skipped stages are released
+      // in order, so this issuer never holds a stage the producer needs for a
+      // later one.
+      int pend = -1, sc = 0, vc = 0;
+      for (int u = 0; u < nkv && ok; ++u) {
+        const int pos_k = pos + 2 * u;
+        if (!plan_uses(p, u, i)) {
+          if (pend >= 0) {
+            if (!flush_pv(pos + 2 * pend + 1, n, vc)) { ok = false; break; }
+            pend = -1;
+          }
+          for (int kind = 0; kind < 2; ++kind) {
+            const int st = acquire(pos_k + kind);
+            if (st < 0) { ok = false; break; }
+            mbar_arrive(b.kv_empty(st));
+          }
+          continue;
+        }
+        const int sk = acquire(pos_k);
+        if (sk < 0 || !issue_s(sk)) { ok = false; break; }
+        if (++sc == n) tc_commit(b.q_empty(i));
+        tc_commit(b.kv_empty(sk));
+        if (pend >= 0 && !flush_pv(pos + 2 * pend + 1, n, vc)) { ok = false; break; }
+        pend = u;
       }
-      pos += 2;
+      if (ok && pend >= 0 && !flush_pv(pos + 2 * pend + 1, n, vc)) ok = false;
+      pos += 2 * nkv;
+      feed_release<BS>(feed, slot);
     }
   }
   if (!ok) record_failure(a, abort_flag, kStatusMma);
@@ -948,7 +1221,7 @@ __device__ __forceinline__ void mma_role_decoupled(const FwdArgs& a, const Bars<
   if (!wait_bounded(b.mma_done(), 0, &never, limit)) atomicOr(a.status, kStatusDrain);
 }
 
-template <int D, int ELEM>
+template <int D, int ELEM, bool BS>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                   const __grid_constant__ CUtensorMap map_v, const FwdArgs a) {
@@ -1000,29 +1273,32 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_holder;
-  const TileFeed feed = make_feed(b, feed_ring);
+  // block-sparse plan slots: two rows, 16-byte aligned, after the barriers
+  const uint32_t plan_addr = sQ + C::PLAN_OFFSET;
+  const TileFeed feed =
+      make_feed<BS>(b, feed_ring, plan_addr, reinterpret_cast<const uint16_t*>(smem_raw + (plan_addr - raw_addr)));
 
   // Each role's code sits inside the branch that set its register budget, so
   // the compiler allocates the softmax code for REG_SOFTMAX registers.
   if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(C::REG_OTHER));
     if (warp == C::LOAD_WARP && lane == 0)
-      producer_role<D, ELEM>(a, b, sQ, sKV, &map_q, &map_k, &map_v, feed, abort_flag);
+      producer_role<D, ELEM, BS>(a, b, sQ, sKV, &map_q, &map_k, &map_v, feed, abort_flag);
     else if (lane == 0) {
       if constexpr (C::DECOUPLED) {
         if (warp == C::MMA_WARP || warp == C::MMA_WARP1)
-          mma_role_decoupled<D, ELEM>(a, b, warp == C::MMA_WARP ? 0 : 1, sQ, sKV, tmem, feed, abort_flag);
+          mma_role_decoupled<D, ELEM, BS>(a, b, warp == C::MMA_WARP ? 0 : 1, sQ, sKV, tmem, feed, abort_flag);
       } else {
-        if (warp == C::MMA_WARP) mma_role<D, ELEM>(a, b, sQ, sKV, tmem, feed, abort_flag);
+        if (warp == C::MMA_WARP) mma_role<D, ELEM, BS>(a, b, sQ, sKV, tmem, feed, abort_flag);
       }
     }
     // the remaining warps of this warpgroup only give their registers away
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(C::REG_SOFTMAX));
     if constexpr (C::DECOUPLED)
-      softmax_role_decoupled<D, ELEM>(a, b, tmem, warp, lane, feed, abort_flag);
+      softmax_role_decoupled<D, ELEM, BS>(a, b, tmem, warp, lane, feed, abort_flag);
     else
-      softmax_role<D, ELEM>(a, b, tmem, warp, lane, feed, abort_flag);
+      softmax_role<D, ELEM, BS>(a, b, tmem, warp, lane, feed, abort_flag);
   }
 
   __syncthreads();

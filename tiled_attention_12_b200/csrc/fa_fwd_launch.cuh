@@ -6,10 +6,12 @@
 
 namespace fa {
 
-template <int D, int ELEM>
+// BS: the block-sparse instantiation (walks l.args->plan); the dense one
+// compiles without any of the plan logic.
+template <int D, int ELEM, bool BS>
 cudaError_t launch_fwd_t(const FwdLaunch& l) {
   using C = FwdCfg<D, ELEM>;
-  auto kernel = fa_fwd_kernel<D, ELEM>;
+  auto kernel = fa_fwd_kernel<D, ELEM, BS>;
   // The attribute is per device; setting it again is harmless.
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;

@@ -23,9 +23,17 @@ struct FwdLaunch {
 cudaError_t launch_fwd_bf16(int d, const FwdLaunch& l);
 cudaError_t launch_fwd_f16(int d, const FwdLaunch& l);
 cudaError_t launch_fwd_e4m3(int d, const FwdLaunch& l);
+// Block-sparse instantiations (args->plan set); called by the three above.
+cudaError_t launch_fwd_sparse(int d, int elem, const FwdLaunch& l);
 cudaError_t launch_quantize_e4m3(const void* x, void* x8, float* scales, int BH, int N, int d,
                                  cudaStream_t stream);
 int fwd_smem_bytes(int d, int elem);
+// Block-sparse plan rows (layout in fa_fwd_kernel.cuh) from a uint8 block
+// mask [BH, ceil(N/128), ceil(N/128)].
+int block_sparse_plan_stride(int N);
+size_t block_sparse_plan_bytes(int BH, int N);
+cudaError_t launch_block_sparse_plan(const uint8_t* mask, uint16_t* plan, int BH, int N, int causal,
+                                     cudaStream_t stream);
 
 struct BwdLaunch {
   CUtensorMap map_q, map_k, map_v, map_do;

@@ -114,3 +114,29 @@ def make_tensor(shape, seed: int, dtype=torch.bfloat16, scale: float = 1.0):
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
     return (torch.randn(shape, generator=g, dtype=torch.float32) * scale).to(dtype)
+
+
+def make_block_mask(B: int, H: int, N: int, kind: str = "random", density: float = 0.5, window: int = 2,
+                    seed: int = 0, block: int = 128) -> torch.Tensor:
+    """Seeded uint8 block mask [B, H, ceil(N/block), ceil(N/block)] (1 = computed).
+
+    kind "random": each block independently with probability ``density``.
+    kind "window": key blocks within ``window`` of the query block plus key
+    block 0 (a sliding window with one global block, the Longformer-style
+    pattern the block-sparse pages describe).
+    kind "ones" / "zeros": every block / none.
+    """
+    nb = (N + block - 1) // block
+    if kind == "ones":
+        return torch.ones((B, H, nb, nb), dtype=torch.uint8)
+    if kind == "zeros":
+        return torch.zeros((B, H, nb, nb), dtype=torch.uint8)
+    if kind == "random":
+        g = torch.Generator().manual_seed(seed)
+        return (torch.rand((B, H, nb, nb), generator=g) < density).to(torch.uint8)
+    if kind == "window":
+        i = torch.arange(nb)[:, None]
+        j = torch.arange(nb)[None, :]
+        m = ((i - j).abs() <= window) | (j == 0)
+        return m.to(torch.uint8).expand(B, H, nb, nb).contiguous()
+    raise ValueError(kind)
