@@ -103,6 +103,25 @@ fa_status fa_fwd_fp8(const void* q8, const float* q_scale, const void* k8, const
                      float softmax_scale, int causal, void* stream);
 
 /*
+ * fa_fwd_strided — fa_fwd on [B, H, N, d] views with arbitrary strides, for
+ * example the (batch, seq, heads, dim) layout, or q, k, v sliced out of one
+ * packed projection.  The last (d) dimension must be contiguous.
+ *   strides : host array of 12 element strides, read during the call:
+ *             {q_b, q_h, q_n, k_b, k_h, k_n, v_b, v_h, v_n, o_b, o_h, o_n};
+ *             element (b, h, n, c) of q is q[b*q_b + h*q_h + n*q_n + c].
+ *             Each must be positive, a multiple of 8 elements (16 bytes; the
+ *             TMA copies and the 16-byte output stores need it) and below
+ *             2^39, else FA_ERR_INVALID.  The caller guarantees that the o
+ *             view does not overlap itself or the inputs.
+ *   lse     : contiguous [B, H, N] fp32 as in fa_fwd, or NULL.
+ *   Other arguments, dtypes and errors as in fa_fwd.  FA_E4M3 quantises the
+ *   strided q and k into contiguous codes in the library workspace.
+ */
+fa_status fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
+                         int B, int H, int N, int d, const long long* strides,
+                         float softmax_scale, int causal, fa_dtype dtype, void* stream);
+
+/*
  * fa_fwd_block_sparse — fa_fwd restricted to chosen 128 x 128 blocks of the
  * attention matrix ("深度解析注意力机制的变体与演进", Block Sparse Attention:
  * the matrix is cut into fixed-size blocks and only some are computed, full

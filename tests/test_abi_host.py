@@ -82,3 +82,22 @@ def test_block_mask_generator_is_seeded_and_shaped():
     assert (a == make_block_mask(2, 3, 1000, "random", 0.4, seed=5)).all()
     w = make_block_mask(1, 1, 1024, "window", window=1)
     assert w[0, 0, 5].tolist() == [1, 0, 0, 0, 1, 1, 1, 0]
+
+
+def test_strided_rejects_bad_strides_without_cuda():
+    L = B.load()
+    f = L.fa_fwd_strided
+    def strides(*vals):
+        return (ctypes.c_longlong * 12)(*vals)
+    ok = [4 * 256 * 64, 256 * 64, 64] * 4
+    assert f(P, P, P, P * 2, None, 1, 4, 256, 64, None, 0.1, 0, 0, None) == B.FA_ERR_INVALID       # no strides
+    bad = list(ok); bad[2] = 60                                                                     # q row stride
+    assert f(P, P, P, P * 2, None, 1, 4, 256, 64, strides(*bad), 0.1, 0, 0, None) == B.FA_ERR_INVALID
+    bad = list(ok); bad[10] = 0                                                                     # o head stride
+    assert f(P, P, P, P * 2, None, 1, 4, 256, 64, strides(*bad), 0.1, 0, 0, None) == B.FA_ERR_INVALID
+    bad = list(ok); bad[6] = -64                                                                    # v batch stride
+    assert f(P, P, P, P * 2, None, 1, 4, 256, 64, strides(*bad), 0.1, 0, 0, None) == B.FA_ERR_INVALID
+    bad = list(ok); bad[4] = 1 << 40                                                                # k too far
+    assert f(P, P, P, P * 2, None, 1, 4, 256, 64, strides(*bad), 0.1, 0, 0, None) == B.FA_ERR_INVALID
+    assert f(P, P, P, P * 2, None, 1, 4, 256, 48, strides(*ok), 0.1, 0, 0, None) == B.FA_ERR_UNSUPPORTED
+    assert f(P, P, P, P, None, 1, 4, 256, 64, strides(*ok), 0.1, 0, 0, None) == B.FA_ERR_INVALID  # o aliases q

@@ -49,13 +49,14 @@ def load():
     L.fa_fwd_e4m3_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
     L.fa_fwd_block_sparse.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, i, vp]
+    L.fa_fwd_strided.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, ctypes.POINTER(ctypes.c_longlong), f, i, i, vp]
     L.fa_last_device_status.argtypes = [vp]
     L.fa_status_string.argtypes = [i]
     L.fa_status_string.restype = ctypes.c_char_p
     L.fa_release.argtypes = []
     L.fa_debug_set_wait_limit.argtypes = [ctypes.c_uint64]
     L.fa_debug_withhold_arrival.argtypes = [i]
-    for name in ("fa_fwd", "fa_bwd", "fa_fwd_block_sparse", "fa_quantize_e4m3", "fa_fwd_fp8",
+    for name in ("fa_fwd", "fa_fwd_strided", "fa_bwd", "fa_fwd_block_sparse", "fa_quantize_e4m3", "fa_fwd_fp8",
                  "fa_fwd_e4m3_noalloc", "fa_last_device_status", "fa_release",
                  "fa_debug_set_wait_limit", "fa_debug_withhold_arrival"):
         getattr(L, name).restype = ctypes.c_int
@@ -96,14 +97,17 @@ def fa_fwd(q, k, v, o=None, lse=None, softmax_scale=None, causal=False, dtype=No
            want_lse=True):
     """Forward pass on [B, H, N, d] CUDA tensors.  Returns (o, lse).
 
-    dtype: None (from q: bf16 or fp16) or FA_E4M3 (q, k bf16, quantised by the
-    library).  Output tensors are allocated when not given.
+    q, k, v may be strided views (for example the (batch, seq, heads, dim)
+    layout seen through ``.transpose(1, 2)``) as long as d is contiguous;
+    those go through fa_fwd_strided.  dtype: None (from q: bf16 or fp16) or
+    FA_E4M3 (q, k 16-bit, quantised by the library).  Output tensors are
+    allocated when not given (o with v's strides).
     """
     import torch
 
     for t in (q, k, v):
-        if not (t.is_cuda and t.is_contiguous() and t.dim() == 4):
-            raise ValueError("q, k, v must be contiguous 4-D CUDA tensors")
+        if not (t.is_cuda and t.dim() == 4):
+            raise ValueError("q, k, v must be 4-D CUDA tensors")
     if q.shape != k.shape or q.shape != v.shape:
         raise ValueError("q, k, v shapes differ")
     B, H, N, d = q.shape
@@ -113,9 +117,18 @@ def fa_fwd(q, k, v, o=None, lse=None, softmax_scale=None, causal=False, dtype=No
     if lse is None and want_lse:
         lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
     scale = (1.0 / d ** 0.5) if softmax_scale is None else float(softmax_scale)
-    st = load().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, scale,
-                       int(bool(causal)), code, _stream(stream))
-    _check(st, "fa_fwd")
+    if all(t.is_contiguous() for t in (q, k, v, o)):
+        st = load().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, scale,
+                           int(bool(causal)), code, _stream(stream))
+        _check(st, "fa_fwd")
+        return o, lse
+    for t in (q, k, v, o):
+        if t.stride(3) != 1:
+            raise ValueError("the last (d) dimension must be contiguous")
+    strides = (ctypes.c_longlong * 12)(*[t.stride(i) for t in (q, k, v, o) for i in range(3)])
+    st = load().fa_fwd_strided(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, strides, scale,
+                               int(bool(causal)), code, _stream(stream))
+    _check(st, "fa_fwd_strided")
     return o, lse
 
 

@@ -139,16 +139,49 @@ int group_heads(int BH, int N, int d, int qk_bytes) {
   return g;
 }
 
+// Element strides of q, k, v and o ([B, H, N, d] views, d contiguous).
+struct Layout {
+  fa::Strides q, k, v, o;
+};
+
+Layout contiguous_layout(int H, int N, int d) {
+  const fa::Strides c = fa::contiguous_strides(H, N, d);
+  return Layout{c, c, c, c};
+}
+
+// A [B, H, N, d] view as a 4-D TMA map {d, N, H, B} at byte strides
+// {n, h, b} * elem_bytes; box {64 (or d) elements of 16 bits | 128 bytes of
+// 8 bits, 128 rows, 1, 1}, swizzled to match the tcgen05 shared-memory layout.
+fa_status make_map4(CUtensorMap* map, const void* ptr, int B, int H, int N, int d, int elem_bytes, bool fp16,
+                    const fa::Strides& st) {
+  const CUtensorMapDataType dt = elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : (fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+  const int row_bytes = d * elem_bytes;
+  const int span = row_bytes >= 128 ? 128 : row_bytes;
+  const CUtensorMapSwizzle sw = span == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(st.n) * elem_bytes, static_cast<cuuint64_t>(st.h) * elem_bytes,
+                           static_cast<cuuint64_t>(st.b) * elem_bytes};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(span / elem_bytes), 128u, 1u, 1u};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = g_encode(map, dt, 4, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_INVALID;
+}
+
 fa_status launch_attention(DeviceState* ds, int elem, const void* q, const void* k, const void* v, void* o,
-                           float* lse, const float* q_scale, const float* k_scale, int BH, int N, int d,
-                           float softmax_scale, int causal, cudaStream_t stream, const uint16_t* plan = nullptr) {
+                           float* lse, const float* q_scale, const float* k_scale, int B, int H, int N, int d,
+                           float softmax_scale, int causal, cudaStream_t stream, const Layout& lay,
+                           const uint16_t* plan = nullptr) {
   fa::FwdLaunch l;
   const int qk_bytes = elem == fa::kElemE4M3 ? 1 : 2;
+  const int BH = B * H;
   fa_status st;
   const bool fp16 = elem == fa::kElemF16;
-  if ((st = make_map(&l.map_q, q, BH, N, d, qk_bytes, fp16)) != FA_OK) return st;
-  if ((st = make_map(&l.map_k, k, BH, N, d, qk_bytes, fp16)) != FA_OK) return st;
-  if ((st = make_map(&l.map_v, v, BH, N, d, 2, fp16)) != FA_OK) return st;
+  if ((st = make_map4(&l.map_q, q, B, H, N, d, qk_bytes, fp16, lay.q)) != FA_OK) return st;
+  if ((st = make_map4(&l.map_k, k, B, H, N, d, qk_bytes, fp16, lay.k)) != FA_OK) return st;
+  if ((st = make_map4(&l.map_v, v, B, H, N, d, 2, fp16, lay.v)) != FA_OK) return st;
   fa::FwdArgs a;
   std::memset(&a, 0, sizeof(a));
   a.o = o;
@@ -158,6 +191,10 @@ fa_status launch_attention(DeviceState* ds, int elem, const void* q, const void*
   a.status = ds->status;
   a.sched = ds->status + 64 + 2 * (ds->next_slot.fetch_add(1u) % kSchedSlots);
   a.BH = BH;
+  a.H = H;
+  a.o_sb = lay.o.b;
+  a.o_sh = lay.o.h;
+  a.o_sn = lay.o.n;
   a.N = N;
   a.n_qpairs = (N + 255) / 256;
   a.n_work = BH * a.n_qpairs;
@@ -197,8 +234,9 @@ struct Quantised {
   float* ks;
 };
 
-fa_status quantise_qk(DeviceState* ds, const void* q, const void* k, int BH, int N, int d, cudaStream_t s,
-                      Quantised* out) {
+fa_status quantise_qk(DeviceState* ds, const void* q, const void* k, int B, int H, int N, int d, const Layout& lay,
+                      cudaStream_t s, Quantised* out) {
+  const int BH = B * H;
   const size_t elems = static_cast<size_t>(BH) * N * d;
   const size_t n_scales = static_cast<size_t>(BH) * ((N + 127) / 128);
   const size_t codes_bytes = (elems + 255) & ~static_cast<size_t>(255);
@@ -212,17 +250,14 @@ fa_status quantise_qk(DeviceState* ds, const void* q, const void* k, int BH, int
   out->k8 = out->q8 + codes_bytes;
   out->qs = reinterpret_cast<float*>(out->k8 + codes_bytes);
   out->ks = out->qs + n_scales;
-  if (fa::launch_quantize_e4m3(q, out->q8, out->qs, BH, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
-  if (fa::launch_quantize_e4m3(k, out->k8, out->ks, BH, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (fa::launch_quantize_e4m3(q, out->q8, out->qs, B, H, N, d, lay.q, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (fa::launch_quantize_e4m3(k, out->k8, out->ks, B, H, N, d, lay.k, s) != cudaSuccess) return FA_ERR_CUDA;
   return FA_OK;
 }
 
-}  // namespace
-
-extern "C" {
-
-fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
-                 float softmax_scale, int causal, fa_dtype dtype, void* stream) {
+// Checks shared by the forward entry points (before any CUDA call).
+fa_status check_forward(const void* q, const void* k, const void* v, void* o, const float* lse, int B, int H, int N,
+                        int d, float softmax_scale, int causal, fa_dtype dtype) {
   if (dtype != FA_BF16 && dtype != FA_FP16 && dtype != FA_E4M3) return FA_ERR_INVALID;
   fa_status st = check_shape(B, H, N, d);
   if (st != FA_OK) return st;
@@ -232,58 +267,82 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     return FA_ERR_INVALID;
   if (!scale_ok(softmax_scale) || (causal != 0 && causal != 1)) return FA_ERR_INVALID;
   if (o == q || o == k || o == v) return FA_ERR_INVALID;
+  return FA_OK;
+}
 
+// The forward for 16-bit inputs, or e4m3 Q/K quantised here first (the codes
+// are contiguous whatever the inputs' strides), optionally block-sparse.
+fa_status forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                  float softmax_scale, int causal, fa_dtype dtype, cudaStream_t s, const Layout& lay,
+                  const uint8_t* block_mask) {
   DeviceState* ds = nullptr;
+  fa_status st;
   if ((st = device_state(&ds)) != FA_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int BH = B * H;
-  if (dtype == FA_BF16) return launch_attention(ds, fa::kElemBF16, q, k, v, o, lse, nullptr, nullptr, BH, N, d,
-                                                softmax_scale, causal, s);
-  if (dtype == FA_FP16) return launch_attention(ds, fa::kElemF16, q, k, v, o, lse, nullptr, nullptr, BH, N, d,
-                                                softmax_scale, causal, s);
-
-  // FA_E4M3: quantise q and k into the library workspace, then attend.
+  uint16_t* plan = nullptr;
+  if (block_mask != nullptr) {
+    {
+      std::lock_guard<std::mutex> lock(g_mu);
+      if ((st = grow(&ds->plan_ws, &ds->plan_ws_bytes, fa::block_sparse_plan_bytes(B * H, N))) != FA_OK) return st;
+      plan = static_cast<uint16_t*>(ds->plan_ws);
+    }
+    if (fa::launch_block_sparse_plan(block_mask, plan, B * H, N, causal, s) != cudaSuccess) return FA_ERR_CUDA;
+  }
+  if (dtype == FA_BF16 || dtype == FA_FP16)
+    return launch_attention(ds, dtype == FA_BF16 ? fa::kElemBF16 : fa::kElemF16, q, k, v, o, lse, nullptr, nullptr, B,
+                            H, N, d, softmax_scale, causal, s, lay, plan);
   Quantised qz;
-  if ((st = quantise_qk(ds, q, k, BH, N, d, s, &qz)) != FA_OK) return st;
-  return launch_attention(ds, fa::kElemE4M3, qz.q8, qz.k8, v, o, lse, qz.qs, qz.ks, BH, N, d, softmax_scale, causal,
-                          s);
+  if ((st = quantise_qk(ds, q, k, B, H, N, d, lay, s, &qz)) != FA_OK) return st;
+  const fa::Strides codes = fa::contiguous_strides(H, N, d);
+  const Layout lay8{codes, codes, lay.v, lay.o};
+  return launch_attention(ds, fa::kElemE4M3, qz.q8, qz.k8, v, o, lse, qz.qs, qz.ks, B, H, N, d, softmax_scale, causal,
+                          s, lay8, plan);
+}
+
+// Strides of one 16-bit [B, H, N, d] view: positive, 16-byte multiples (the
+// TMA copies and the 16-byte output stores need that), below 2^39 elements.
+bool strides_ok(const fa::Strides& st) {
+  const long long lim = 1LL << 39;
+  for (long long x : {st.b, st.h, st.n})
+    if (x <= 0 || x % 8 != 0 || x >= lim) return false;
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                 float softmax_scale, int causal, fa_dtype dtype, void* stream) {
+  fa_status st = check_forward(q, k, v, o, lse, B, H, N, d, softmax_scale, causal, dtype);
+  if (st != FA_OK) return st;
+  return forward(q, k, v, o, lse, B, H, N, d, softmax_scale, causal, dtype, static_cast<cudaStream_t>(stream),
+                 contiguous_layout(H, N, d), nullptr);
+}
+
+fa_status fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                         const long long* strides, float softmax_scale, int causal, fa_dtype dtype, void* stream) {
+  fa_status st = check_forward(q, k, v, o, lse, B, H, N, d, softmax_scale, causal, dtype);
+  if (st != FA_OK) return st;
+  if (strides == nullptr) return FA_ERR_INVALID;
+  Layout lay;
+  fa::Strides* views[4] = {&lay.q, &lay.k, &lay.v, &lay.o};
+  for (int t = 0; t < 4; ++t) {
+    *views[t] = fa::Strides{strides[3 * t], strides[3 * t + 1], strides[3 * t + 2]};
+    if (!strides_ok(*views[t])) return FA_ERR_INVALID;
+  }
+  return forward(q, k, v, o, lse, B, H, N, d, softmax_scale, causal, dtype, static_cast<cudaStream_t>(stream), lay,
+                 nullptr);
 }
 
 fa_status fa_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
                               int d, float softmax_scale, int causal, const uint8_t* block_mask, fa_dtype dtype,
                               void* stream) {
-  if (dtype != FA_BF16 && dtype != FA_FP16 && dtype != FA_E4M3) return FA_ERR_INVALID;
-  fa_status st = check_shape(B, H, N, d);
+  fa_status st = check_forward(q, k, v, o, lse, B, H, N, d, softmax_scale, causal, dtype);
   if (st != FA_OK) return st;
-  if (dtype == FA_E4M3 && d != 128) return FA_ERR_UNSUPPORTED;
   if ((N + 127) / 128 > fa::kPlanMaxTiles) return FA_ERR_UNSUPPORTED;
-  if (!q || !k || !v || !o || !block_mask) return FA_ERR_INVALID;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)))
-    return FA_ERR_INVALID;
-  if (!scale_ok(softmax_scale) || (causal != 0 && causal != 1)) return FA_ERR_INVALID;
-  if (o == q || o == k || o == v) return FA_ERR_INVALID;
-
-  DeviceState* ds = nullptr;
-  if ((st = device_state(&ds)) != FA_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int BH = B * H;
-  uint16_t* plan = nullptr;
-  {
-    std::lock_guard<std::mutex> lock(g_mu);
-    if ((st = grow(&ds->plan_ws, &ds->plan_ws_bytes, fa::block_sparse_plan_bytes(BH, N))) != FA_OK) return st;
-    plan = static_cast<uint16_t*>(ds->plan_ws);
-  }
-  if (fa::launch_block_sparse_plan(block_mask, plan, BH, N, causal, s) != cudaSuccess) return FA_ERR_CUDA;
-  if (dtype == FA_BF16)
-    return launch_attention(ds, fa::kElemBF16, q, k, v, o, lse, nullptr, nullptr, BH, N, d, softmax_scale, causal, s,
-                            plan);
-  if (dtype == FA_FP16)
-    return launch_attention(ds, fa::kElemF16, q, k, v, o, lse, nullptr, nullptr, BH, N, d, softmax_scale, causal, s,
-                            plan);
-  Quantised qz;
-  if ((st = quantise_qk(ds, q, k, BH, N, d, s, &qz)) != FA_OK) return st;
-  return launch_attention(ds, fa::kElemE4M3, qz.q8, qz.k8, v, o, lse, qz.qs, qz.ks, BH, N, d, softmax_scale, causal,
-                          s, plan);
+  if (!block_mask) return FA_ERR_INVALID;
+  return forward(q, k, v, o, lse, B, H, N, d, softmax_scale, causal, dtype, static_cast<cudaStream_t>(stream),
+                 contiguous_layout(H, N, d), block_mask);
 }
 
 fa_status fa_quantize_e4m3(const void* x, void* x8, float* scales, int B, int H, int N, int d, void* stream) {
@@ -293,7 +352,8 @@ fa_status fa_quantize_e4m3(const void* x, void* x8, float* scales, int B, int H,
   if (!aligned16(x) || !aligned16(x8) || !aligned16(scales)) return FA_ERR_INVALID;
   DeviceState* ds = nullptr;
   if ((st = device_state(&ds)) != FA_OK) return st;
-  return map_cuda(fa::launch_quantize_e4m3(x, x8, scales, B * H, N, d, static_cast<cudaStream_t>(stream)));
+  return map_cuda(fa::launch_quantize_e4m3(x, x8, scales, B, H, N, d, fa::contiguous_strides(H, N, d),
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 fa_status fa_fwd_fp8(const void* q8, const float* q_scale, const void* k8, const float* k_scale, const void* v,
@@ -311,8 +371,8 @@ fa_status fa_fwd_fp8(const void* q8, const float* q_scale, const void* k8, const
   if (o == q8 || o == k8 || o == v) return FA_ERR_INVALID;
   DeviceState* ds = nullptr;
   if ((st = device_state(&ds)) != FA_OK) return st;
-  return launch_attention(ds, fa::kElemE4M3, q8, k8, v, o, lse, q_scale, k_scale, B * H, N, d, softmax_scale,
-                          causal, static_cast<cudaStream_t>(stream));
+  return launch_attention(ds, fa::kElemE4M3, q8, k8, v, o, lse, q_scale, k_scale, B, H, N, d, softmax_scale, causal,
+                          static_cast<cudaStream_t>(stream), contiguous_layout(H, N, d));
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,

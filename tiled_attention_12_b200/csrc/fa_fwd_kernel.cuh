@@ -78,7 +78,7 @@ constexpr int kPlanSlotBytes = 2 * (kPlanHeader + 3 * kPlanMaxTiles);
 static_assert(kPlanSlotBytes % 16 == 0, "plan slots must be whole 16-byte units");
 
 struct FwdArgs {
-  void* o;                 // [BH, N, D], element type of V
+  void* o;                 // [B, H, N, D] at the strides below, element type of V
   float* lse;              // [BH, N] fp32 or nullptr
   const float* q_scale;    // [BH, ceil(N/128)] (e4m3 only)
   const float* k_scale;    // [BH, ceil(N/128)] (e4m3 only)
@@ -97,7 +97,16 @@ struct FwdArgs {
   const uint16_t* plan;    // block-sparse plan rows [n_work][plan_row] or nullptr (dense)
   int plan_stride;         // entries per list in a plan row
   int plan_row_bytes;      // bytes per plan row (2 * (8 + 3 * plan_stride))
+  int H;                   // heads: bh = b * H + h
+  long long o_sb, o_sh, o_sn;  // O strides in elements (batch, head, row); D is contiguous
 };
+
+// Start of output row `row` of head bh.
+template <typename T>
+__device__ __forceinline__ T* o_row(const FwdArgs& a, int bh, int row) {
+  const int b = bh / a.H, h = bh - b * a.H;
+  return reinterpret_cast<T*>(a.o) + b * a.o_sb + h * a.o_sh + row * a.o_sn;
+}
 
 template <int D, int ELEM>
 struct FwdCfg {
@@ -403,6 +412,7 @@ __device__ __forceinline__ void producer_role(const FwdArgs& a, const Bars<FwdCf
     }
     const Plan p = make_plan<BS>(a, t, feed, slot);
     const int n0 = p.n0, n1 = p.n1;
+    const int tb = t.bh / a.H, th = t.bh - tb * a.H;  // tensor-map coordinates of the head
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const int n = i ? n1 : n0;
@@ -415,8 +425,8 @@ __device__ __forceinline__ void producer_role(const FwdArgs& a, const Bars<FwdCf
       mbar_arrive_expect_tx(b.q_full(i), C::Q_TILE);
 #pragma unroll
       for (int c = 0; c < C::QK_ROW / C::SW_QK; ++c)
-        tma_load_3d(sQ + i * C::Q_TILE + c * C::BM * C::SW_QK, map_q, b.q_full(i), c * (C::SW_QK / C::QK_BYTES),
-                    q0 + i * 128, t.bh);
+        tma_load_4d(sQ + i * C::Q_TILE + c * C::BM * C::SW_QK, map_q, b.q_full(i), c * (C::SW_QK / C::QK_BYTES),
+                    q0 + i * 128, th, tb);
       ++use;
     }
     for (int u = 0; ok && u < p.nkv; ++u) {
@@ -438,13 +448,13 @@ __device__ __forceinline__ void producer_role(const FwdArgs& a, const Bars<FwdCf
           mbar_arrive_expect_tx(b.kv_full(s), C::K_TILE);
 #pragma unroll
           for (int c = 0; c < C::QK_ROW / C::SW_QK; ++c)
-            tma_load_3d(dst + c * C::BN * C::SW_QK, map_k, b.kv_full(s), c * (C::SW_QK / C::QK_BYTES), j * 128,
-                        t.bh);
+            tma_load_4d(dst + c * C::BN * C::SW_QK, map_k, b.kv_full(s), c * (C::SW_QK / C::QK_BYTES), j * 128,
+                        th, tb);
         } else {
           mbar_arrive_expect_tx(b.kv_full(s), C::V_TILE);
 #pragma unroll
           for (int c = 0; c < C::V_ROW / C::SW_V; ++c)
-            tma_load_3d(dst + c * C::BN * C::SW_V, map_v, b.kv_full(s), c * (C::SW_V / 2), j * 128, t.bh);
+            tma_load_4d(dst + c * C::BN * C::SW_V, map_v, b.kv_full(s), c * (C::SW_V / 2), j * 128, th, tb);
         }
       }
     }
@@ -810,7 +820,7 @@ template <int D, int ELEM>
 __device__ __forceinline__ void epilogue_row(const FwdArgs& a, uint32_t t_o, int bh, int qrow, float m, float l) {
   using OutT = typename std::conditional<ELEM == kElemF16, __half, __nv_bfloat16>::type;
   const float inv_l = 1.f / l;
-  OutT* orow = reinterpret_cast<OutT*>(a.o) + (static_cast<size_t>(bh) * a.N + qrow) * D;
+  OutT* orow = o_row<OutT>(a, bh, qrow);
 #pragma unroll
   for (int c = 0; c < D / 32; ++c) {
     uint32_t orr[32];
@@ -839,7 +849,7 @@ template <int D, int ELEM>
 __device__ __forceinline__ void empty_row(const FwdArgs& a, int bh, int qrow) {
   if (qrow >= a.N) return;
   using OutT = typename std::conditional<ELEM == kElemF16, __half, __nv_bfloat16>::type;
-  uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<OutT*>(a.o) + (static_cast<size_t>(bh) * a.N + qrow) * D);
+  uint4* dst = reinterpret_cast<uint4*>(o_row<OutT>(a, bh, qrow));
 #pragma unroll
   for (int v = 0; v < D * 2 / 16; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
   if (a.lse != nullptr) a.lse[static_cast<size_t>(bh) * a.N + qrow] = -INFINITY;

@@ -12,6 +12,14 @@ namespace fa {
 struct FwdArgs;
 struct BwdArgs;
 
+// Element strides of a [B, H, N, d] tensor whose last dimension is contiguous.
+struct Strides {
+  long long b, h, n;
+};
+inline Strides contiguous_strides(int H, int N, int d) {
+  return Strides{static_cast<long long>(H) * N * d, static_cast<long long>(N) * d, d};
+}
+
 struct FwdLaunch {
   CUtensorMap map_q, map_k, map_v;
   const FwdArgs* args;
@@ -25,8 +33,10 @@ cudaError_t launch_fwd_f16(int d, const FwdLaunch& l);
 cudaError_t launch_fwd_e4m3(int d, const FwdLaunch& l);
 // Block-sparse instantiations (args->plan set); called by the three above.
 cudaError_t launch_fwd_sparse(int d, int elem, const FwdLaunch& l);
-cudaError_t launch_quantize_e4m3(const void* x, void* x8, float* scales, int BH, int N, int d,
-                                 cudaStream_t stream);
+// e4m3 codes [B*H, N, d] (contiguous) and per-128-row-tile scales of a
+// 16-bit input read at strides `st`.
+cudaError_t launch_quantize_e4m3(const void* x, void* x8, float* scales, int B, int H, int N, int d,
+                                 const Strides& st, cudaStream_t stream);
 int fwd_smem_bytes(int d, int elem);
 // Block-sparse plan rows (layout in fa_fwd_kernel.cuh) from a uint8 block
 // mask [BH, ceil(N/128), ceil(N/128)].

@@ -92,16 +92,16 @@ fa_status noalloc_setup(NoAllocDevice** out) {
   return FA_OK;
 }
 
-// [BH, N, 128] tensor as a 3-D TMA map with a 128-byte swizzled box of 128
-// rows (the geometry the forward kernel's shared-memory layout expects).
-fa_status noalloc_map(CUtensorMap* map, const void* ptr, int BH, int N, bool codes) {
+// Contiguous [B, H, N, 128] tensor as the forward kernel's 4-D TMA map
+// {d, N, H, B} with a 128-byte swizzled box of 128 rows.
+fa_status noalloc_map(CUtensorMap* map, const void* ptr, int B, int H, int N, bool codes) {
   const int elem = codes ? 1 : 2;
-  const int row_bytes = 128 * elem;
-  cuuint64_t dims[3] = {128u, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(row_bytes) * N};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem), 128u, 1u};
-  cuuint32_t estr[3] = {1u, 1u, 1u};
-  CUresult r = g_na_encode(map, codes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+  const cuuint64_t row_bytes = 128u * elem;
+  cuuint64_t dims[4] = {128u, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {row_bytes, row_bytes * N, row_bytes * N * H};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / elem), 128u, 1u, 1u};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = g_na_encode(map, codes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
                            const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -139,13 +139,14 @@ extern "C" fa_status fa_fwd_e4m3_noalloc(const void* q, const void* k, const voi
   // The quantiser writes every code and scale the attention kernel reads, so
   // nothing left over from an earlier call is ever consumed.
   const int bh = static_cast<int>(BH);
-  if (fa::launch_quantize_e4m3(q, q8, qs, bh, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
-  if (fa::launch_quantize_e4m3(k, k8, ks, bh, N, d, s) != cudaSuccess) return FA_ERR_CUDA;
+  const fa::Strides cont = fa::contiguous_strides(H, N, d);
+  if (fa::launch_quantize_e4m3(q, q8, qs, B, H, N, d, cont, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (fa::launch_quantize_e4m3(k, k8, ks, B, H, N, d, cont, s) != cudaSuccess) return FA_ERR_CUDA;
 
   fa::FwdLaunch l;
-  if ((st = noalloc_map(&l.map_q, q8, bh, N, true)) != FA_OK) return st;
-  if ((st = noalloc_map(&l.map_k, k8, bh, N, true)) != FA_OK) return st;
-  if ((st = noalloc_map(&l.map_v, v, bh, N, false)) != FA_OK) return st;
+  if ((st = noalloc_map(&l.map_q, q8, B, H, N, true)) != FA_OK) return st;
+  if ((st = noalloc_map(&l.map_k, k8, B, H, N, true)) != FA_OK) return st;
+  if ((st = noalloc_map(&l.map_v, v, B, H, N, false)) != FA_OK) return st;
   fa::FwdArgs a;
   std::memset(&a, 0, sizeof(a));
   a.o = o;
@@ -158,6 +159,10 @@ extern "C" fa_status fa_fwd_e4m3_noalloc(const void* q, const void* k, const voi
     a.sched = reinterpret_cast<unsigned int*>(dev->scratch + kSchedOffset) + 2 * (dev->next_slot++ % kSchedSlots);
   }
   a.BH = bh;
+  a.H = H;
+  a.o_sb = cont.b;
+  a.o_sh = cont.h;
+  a.o_sn = cont.n;
   a.N = N;
   a.n_qpairs = (N + 255) / 256;
   a.n_work = bh * a.n_qpairs;

@@ -33,19 +33,28 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
   return r;
 }
 
-__global__ void __launch_bounds__(256) quantize_e4m3_kernel(const uint4* __restrict__ x, uint2* __restrict__ x8,
-                                                            float* __restrict__ scales, int N, int d,
-                                                            int n_tiles) {
+// x is read at element strides (batch, head, row); its rows are contiguous.
+// The codes are written contiguously as [B*H, N, d].
+__global__ void __launch_bounds__(256) quantize_e4m3_kernel(const uint16_t* __restrict__ x, uint2* __restrict__ x8,
+                                                            float* __restrict__ scales, int H, int N, int d,
+                                                            int n_tiles, int vec_shift, long long sb, long long sh,
+                                                            long long sn) {
   const int t = blockIdx.x % n_tiles;
   const int bh = blockIdx.x / n_tiles;
+  const int b = bh / H, h = bh - b * H;
   const int r0 = t * 128;
   const int rows = (N - r0) < 128 ? (N - r0) : 128;
   const size_t vec0 = ((static_cast<size_t>(bh) * N + r0) * d) / 8;  // 8 elements per vector
   const int n_vec = rows * d / 8;
-
+  const uint16_t* tile = x + b * sb + h * sh + r0 * sn;
+  const int vec_mask = (1 << vec_shift) - 1;  // vectors per row - 1
+  // the 16-byte vector v of the tile: row v >> vec_shift, column vector v & vec_mask
+  auto load = [&](int v) {
+    return *reinterpret_cast<const uint4*>(tile + (v >> vec_shift) * sn + (v & vec_mask) * 8);
+  };
   float amax = 0.f;
   for (int v = threadIdx.x; v < n_vec; v += 256) {
-    const uint4 u = x[vec0 + v];
+    const uint4 u = load(v);
     amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(u.x)), fabsf(bf16_hi(u.x))),
                              fmaxf(fabsf(bf16_lo(u.y)), fabsf(bf16_hi(u.y)))));
     amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(u.z)), fabsf(bf16_hi(u.z))),
@@ -62,7 +71,7 @@ __global__ void __launch_bounds__(256) quantize_e4m3_kernel(const uint4* __restr
   const float sc = amax > 0.f ? __fdiv_rn(448.0f, amax) : 1.0f;
 
   for (int v = threadIdx.x; v < n_vec; v += 256) {
-    const uint4 u = x[vec0 + v];
+    const uint4 u = load(v);
     const uint32_t c0 = cvt_e4m3x2(__fmul_rn(bf16_lo(u.x), sc), __fmul_rn(bf16_hi(u.x), sc));
     const uint32_t c1 = cvt_e4m3x2(__fmul_rn(bf16_lo(u.y), sc), __fmul_rn(bf16_hi(u.y), sc));
     const uint32_t c2 = cvt_e4m3x2(__fmul_rn(bf16_lo(u.z), sc), __fmul_rn(bf16_hi(u.z), sc));
@@ -74,13 +83,15 @@ __global__ void __launch_bounds__(256) quantize_e4m3_kernel(const uint4* __restr
 
 }  // namespace
 
-cudaError_t launch_quantize_e4m3(const void* x, void* x8, float* scales, int BH, int N, int d,
-                                 cudaStream_t stream) {
+cudaError_t launch_quantize_e4m3(const void* x, void* x8, float* scales, int B, int H, int N, int d,
+                                 const Strides& st, cudaStream_t stream) {
   const int n_tiles = (N + 127) / 128;
-  const long long blocks = static_cast<long long>(n_tiles) * BH;
+  const long long blocks = static_cast<long long>(n_tiles) * B * H;
   if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
-  quantize_e4m3_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(static_cast<const uint4*>(x), static_cast<uint2*>(x8), scales,
-                                                  N, d, n_tiles);
+  const int vec_shift = d == 32 ? 2 : (d == 64 ? 3 : 4);  // log2(d / 8) vectors per row
+  if ((8 << vec_shift) != d) return cudaErrorInvalidValue;
+  quantize_e4m3_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+      static_cast<const uint16_t*>(x), static_cast<uint2*>(x8), scales, H, N, d, n_tiles, vec_shift, st.b, st.h, st.n);
   return cudaGetLastError();
 }
 
