@@ -163,6 +163,27 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  float softmax_scale, int causal, fa_dtype dtype, void* stream);
 
 /*
+ * fa_merge_partial — folds one partial attention result into accumulators:
+ * the step of ring (sequence-parallel) attention that combines the outputs
+ * of one query block against different key/value blocks
+ * ("深度解析注意力机制的变体与演进", Ring Attention; the combination is the
+ * online-softmax renormalisation of "从理论到实现…" §2.1 applied to blocks):
+ *     LSE = log(exp(LSE_acc) + exp(LSE_part))
+ *     O   = exp(LSE_acc - LSE) O_acc + exp(LSE_part - LSE) O_part
+ * A side with LSE = -inf contributes nothing (both: O = 0, LSE = -inf).
+ *   o_part   : [rows, d] 16-bit (dtype FA_BF16 or FA_FP16), e.g. fa_fwd's o
+ *   lse_part : [rows] fp32 (natural log), e.g. fa_fwd's lse
+ *   o_acc    : [rows, d] fp32 accumulator; lse_acc : [rows] fp32
+ *   first    : 1 = start the accumulation (copy the partial in), 0 = merge
+ *   o_out    : NULL, or [rows, d] 16-bit: write the merged rows there instead
+ *              of into o_acc (the last step); lse_acc is updated either way.
+ * rows = B * H * n for [B, H, n, d] tensors.  All device pointers; o_part,
+ * o_acc and o_out 16-byte aligned.  Asynchronous on `stream`.
+ */
+fa_status fa_merge_partial(const void* o_part, const float* lse_part, float* o_acc, float* lse_acc,
+                           void* o_out, long long rows, int d, fa_dtype dtype, int first, void* stream);
+
+/*
  * fa_last_device_status — synchronises `stream`, reads and clears the device
  * status word of the current device.  FA_OK when no kernel on this device
  * gave up on a wait since the last call; FA_ERR_TIMEOUT otherwise.

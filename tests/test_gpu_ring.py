@@ -1,0 +1,89 @@
+"""GPU checks of ring attention's pieces: the merge kernel (fa_merge_partial)
+against the oracle merge, and the whole ring emulated on one GPU (every
+rank's steps in turn, no rank waiting on another) against plain attention."""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import tiled_attention_12_b200 as fa
+from oracle import attention_ref, attention_rows, merge_partials_ref
+from parity_util import TOL_16, gate, half_ulp, sample_rows
+from tiled_attention_12_b200.ring import ring_attention_emulated
+from tiled_attention_12_b200.synth import Case, make_qkv
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _partials(rows, d, seed, dtype):
+    g = torch.Generator().manual_seed(seed)
+    o_part = torch.randn((rows, d), generator=g).to(dtype)
+    lse_part = torch.randn(rows, generator=g) * 3
+    o_acc = torch.randn((rows, d), generator=g)
+    lse_acc = torch.randn(rows, generator=g) * 3
+    lse_part[::7] = -float("inf")        # empty partial rows
+    lse_acc[::11] = -float("inf")        # empty accumulator rows (77, 154, ... both)
+    o_part[::7] = 0
+    return o_part, lse_part, o_acc, lse_acc
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("d", [32, 64, 128])
+def test_merge_kernel_against_oracle(d, dtype):
+    rows = 1000
+    o_part, lse_part, o_acc, lse_acc = _partials(rows, d, d, dtype)
+    ro, rl = merge_partials_ref(o_acc, lse_acc, o_part, lse_part)
+    acc, la = o_acc.to(DEV), lse_acc.to(DEV)
+    fa.fa_merge_partial(o_part.to(DEV), lse_part.to(DEV), acc, la)
+    torch.cuda.synchronize()
+    acc, la = acc.cpu().double().numpy(), la.cpu().double().numpy()
+    assert np.array_equal(np.isneginf(la), np.isneginf(rl))
+    fin = np.isfinite(rl)
+    assert np.max(np.abs(la[fin] - rl[fin])) <= 1e-5
+    assert np.max(np.abs(acc - ro)) <= 1e-5 * (1 + np.abs(ro).max())
+    # last step: the merged rows go to a 16-bit output, rounded once
+    out = torch.empty((rows, d), device=DEV, dtype=dtype)
+    acc2, la2 = o_acc.to(DEV), lse_acc.to(DEV)
+    fa.fa_merge_partial(o_part.to(DEV), lse_part.to(DEV), acc2, la2, o_out=out)
+    torch.cuda.synchronize()
+    err = np.abs(out.cpu().double().numpy() - ro)
+    assert np.all(err <= half_ulp(ro, dtype) + 1e-5 * (1 + np.abs(ro)))
+    assert torch.equal(acc2.cpu(), o_acc)            # o_acc untouched when o_out is given
+
+
+def test_merge_first_copies():
+    o_part, lse_part, _, _ = _partials(300, 64, 1, torch.bfloat16)
+    acc = torch.full((300, 64), 5.0, device=DEV)
+    la = torch.full((300,), 5.0, device=DEV)
+    fa.fa_merge_partial(o_part.to(DEV), lse_part.to(DEV), acc, la, first=True)
+    torch.cuda.synchronize()
+    assert torch.equal(acc.cpu(), o_part.float()) and torch.equal(la.cpu(), lse_part)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("d", [32, 64, 128])
+def test_emulated_ring_against_oracle(d, world, causal):
+    case = Case("ring", 1, 4, 2048, d, causal, seed=d + world)
+    q, k, v = make_qkv(case)
+    o, lse = ring_attention_emulated(q.to(DEV), k.to(DEV), v.to(DEV), world, causal)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status() == 0
+    ro, rl = attention_ref(q, k, v, case.softmax_scale, causal)
+    gate(o, ro, lse, rl, tol=TOL_16, what=f"ring d{d} w{world} c{causal}")
+
+
+def test_emulated_ring_long_sequence():
+    """B1 H8 N32768 d128 causal over 8 emulated ranks, sampled rows."""
+    case = Case("ring_long", 1, 8, 32768, 128, True, seed=5)
+    q, k, v = make_qkv(case)
+    o, lse = ring_attention_emulated(q.to(DEV), k.to(DEV), v.to(DEV), 8, True)
+    torch.cuda.synchronize()
+    rows = sample_rows(case.N, seed=1, n_random=48)
+    idx = torch.as_tensor(rows, device=DEV)
+    for h in (0, 7):
+        ro, rl = attention_rows(q, k, v, case.softmax_scale, True, 0, h, rows)
+        gate(o[0, h][idx], ro, lse[0, h][idx], rl, tol=TOL_16, what=f"long ring head {h}")

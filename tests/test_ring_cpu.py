@@ -1,0 +1,93 @@
+"""The ring attention schedule and transfers on CPU: gloo ranks run
+ring_attention with the oracle standing in for the two GPU calls (attention
+of one block, merge of one partial), and every rank's rows must equal plain
+attention over the whole sequence."""
+
+from __future__ import annotations
+
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+from tiled_attention_12_b200.ring import ring_steps
+
+
+def test_ring_steps_visit_every_block_once():
+    for world in (1, 2, 3, 8):
+        for rank in range(world):
+            srcs = [s for s, _ in ring_steps(rank, world, False)]
+            assert sorted(srcs) == list(range(world)) and srcs[0] == rank
+            assert all(m == "full" for _, m in ring_steps(rank, world, False))
+            for src, mode in ring_steps(rank, world, True):
+                assert mode == ("full" if src < rank else "causal" if src == rank else "skip")
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _attend_cpu(q, k, v, causal, scale):
+    from oracle import attention_ref
+
+    o, lse = attention_ref(q, k, v, scale, causal, workers=1)
+    return torch.from_numpy(o).to(q.dtype), torch.from_numpy(lse).to(torch.float32)
+
+
+def _merge_cpu(o_part, lse_part, o_acc, lse_acc, o_out, first):
+    from oracle import merge_partials_ref
+
+    if first:
+        o, lse = o_part.double().numpy(), lse_part.double().numpy()
+    else:
+        o, lse = merge_partials_ref(o_acc, lse_acc, o_part, lse_part)
+    lse_acc.copy_(torch.from_numpy(np.asarray(lse)))
+    (o_out if o_out is not None else o_acc).copy_(torch.from_numpy(np.asarray(o)))
+
+
+def _rank(rank, world, causal, port, out):
+    import torch.distributed as dist
+
+    from oracle import attention_ref
+    from tiled_attention_12_b200.ring import ring_attention
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        B, H, n, d = 1, 2, 8, 4
+        g = torch.Generator().manual_seed(3)
+        q, k, v = (torch.randn((B, H, n * world, d), generator=g) for _ in range(3))
+        sl = slice(rank * n, (rank + 1) * n)
+        o, lse = ring_attention(q[:, :, sl].contiguous(), k[:, :, sl].contiguous(), v[:, :, sl].contiguous(),
+                                causal=causal, softmax_scale=0.5, attend=_attend_cpu, merge=_merge_cpu)
+        ro, rl = attention_ref(q, k, v, 0.5, causal, workers=1)
+        out.put((rank, float(np.abs(o.double().numpy() - ro[:, :, sl]).max()),
+                 float(np.abs(lse.double().numpy() - rl[:, :, sl]).max())))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("world", [2, 3])
+def test_gloo_ring_equals_plain_attention(world, causal):
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, world, causal, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+    assert all(p.exitcode == 0 for p in procs)
+    got = sorted(out.get(timeout=10) for _ in range(world))
+    assert [g[0] for g in got] == list(range(world))
+    for _, o_err, l_err in got:
+        assert o_err < 1e-5 and l_err < 1e-5

@@ -49,6 +49,7 @@ def load():
     L.fa_fwd_e4m3_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
     L.fa_fwd_block_sparse.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, i, vp]
+    L.fa_merge_partial.argtypes = [vp, vp, vp, vp, vp, ctypes.c_longlong, i, i, i, vp]
     L.fa_fwd_strided.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, ctypes.POINTER(ctypes.c_longlong), f, i, i, vp]
     L.fa_last_device_status.argtypes = [vp]
     L.fa_status_string.argtypes = [i]
@@ -56,7 +57,7 @@ def load():
     L.fa_release.argtypes = []
     L.fa_debug_set_wait_limit.argtypes = [ctypes.c_uint64]
     L.fa_debug_withhold_arrival.argtypes = [i]
-    for name in ("fa_fwd", "fa_fwd_strided", "fa_bwd", "fa_fwd_block_sparse", "fa_quantize_e4m3", "fa_fwd_fp8",
+    for name in ("fa_fwd", "fa_fwd_strided", "fa_merge_partial", "fa_bwd", "fa_fwd_block_sparse", "fa_quantize_e4m3", "fa_fwd_fp8",
                  "fa_fwd_e4m3_noalloc", "fa_last_device_status", "fa_release",
                  "fa_debug_set_wait_limit", "fa_debug_withhold_arrival"):
         getattr(L, name).restype = ctypes.c_int
@@ -158,6 +159,27 @@ def fa_fwd_block_sparse(q, k, v, block_mask, o=None, lse=None, softmax_scale=Non
                                     int(bool(causal)), _ptr(block_mask), code, _stream(stream))
     _check(st, "fa_fwd_block_sparse")
     return o, lse
+
+
+def fa_merge_partial(o_part, lse_part, o_acc, lse_acc, o_out=None, first=False, stream=None):
+    """Fold a partial result (o_part [..., d] 16-bit, lse_part [...]) into the
+    fp32 accumulators o_acc / lse_acc; with o_out the merged rows go there in
+    16 bits instead.  Returns (o_out or o_acc, lse_acc)."""
+    import torch
+
+    d = o_part.shape[-1]
+    rows = lse_part.numel()
+    for t, dt in ((o_part, None), (lse_part, torch.float32), (o_acc, torch.float32), (lse_acc, torch.float32)):
+        if not (t.is_cuda and t.is_contiguous()) or (dt is not None and t.dtype != dt):
+            raise ValueError("merge operands must be contiguous CUDA tensors (lse and accumulators fp32)")
+    if o_part.numel() != rows * d or o_acc.numel() != rows * d or lse_acc.numel() != rows:
+        raise ValueError("merge operand sizes differ")
+    if o_out is not None and not (o_out.is_contiguous() and o_out.numel() == rows * d and o_out.dtype == o_part.dtype):
+        raise ValueError("o_out must be contiguous, of o_part's size and dtype")
+    st = load().fa_merge_partial(_ptr(o_part), _ptr(lse_part), _ptr(o_acc), _ptr(lse_acc), _ptr(o_out), rows, d,
+                                 _dtype_code(o_part), int(bool(first)), _stream(stream))
+    _check(st, "fa_merge_partial")
+    return (o_out if o_out is not None else o_acc), lse_acc
 
 
 def fa_bwd(q, k, v, o, lse, dout, dq=None, dk=None, dv=None, softmax_scale=None, causal=False, stream=None):

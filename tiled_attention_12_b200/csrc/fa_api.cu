@@ -375,6 +375,22 @@ fa_status fa_fwd_fp8(const void* q8, const float* q_scale, const void* k8, const
                           static_cast<cudaStream_t>(stream), contiguous_layout(H, N, d));
 }
 
+fa_status fa_merge_partial(const void* o_part, const float* lse_part, float* o_acc, float* lse_acc, void* o_out,
+                           long long rows, int d, fa_dtype dtype, int first, void* stream) {
+  if (rows <= 0 || (first != 0 && first != 1)) return FA_ERR_INVALID;
+  if (d != 32 && d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (dtype != FA_BF16 && dtype != FA_FP16) return dtype == FA_E4M3 ? FA_ERR_UNSUPPORTED : FA_ERR_INVALID;
+  if (!o_part || !lse_part || !o_acc || !lse_acc) return FA_ERR_INVALID;
+  if (!aligned16(o_part) || !aligned16(o_acc) || (o_out && !aligned16(o_out))) return FA_ERR_INVALID;
+  if ((reinterpret_cast<uintptr_t>(lse_part) & 3u) || (reinterpret_cast<uintptr_t>(lse_acc) & 3u))
+    return FA_ERR_INVALID;
+  DeviceState* ds = nullptr;
+  fa_status st;
+  if ((st = device_state(&ds)) != FA_OK) return st;
+  return map_cuda(fa::launch_merge_partial(o_part, lse_part, o_acc, lse_acc, o_out, rows, d, dtype == FA_FP16, first,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
                  void* dq, void* dk, void* dv, int B, int H, int N, int d, float softmax_scale, int causal,
                  fa_dtype dtype, void* stream) {

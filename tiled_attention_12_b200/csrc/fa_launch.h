@@ -45,6 +45,11 @@ size_t block_sparse_plan_bytes(int BH, int N);
 cudaError_t launch_block_sparse_plan(const uint8_t* mask, uint16_t* plan, int BH, int N, int causal,
                                      cudaStream_t stream);
 
+// One partial attention result folded into fp32 accumulators (o_out set:
+// the merged rows are written there in 16 bits instead of into o_acc).
+cudaError_t launch_merge_partial(const void* o_part, const float* lse_part, float* o_acc, float* lse_acc, void* o_out,
+                                 long long rows, int d, bool f16, int first, cudaStream_t stream);
+
 struct BwdLaunch {
   CUtensorMap map_q, map_k, map_v, map_do;
   const BwdArgs* args;
