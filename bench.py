@@ -372,6 +372,31 @@ def run_ours(args, rank, world, local_rank):
                 del q, k, v, o, lse, mask
             except Exception as e:  # report, never hide
                 suite[name] = {"error": str(e)[:200]}
+        # full FP8 (FA_E4M3_ALL: Q, K, V and P in e4m3) on the FP8 config's shape
+        fc = WORKLOADS["fp8_b2h16n16384d128_causal"].cases[0]
+        name = "fp8all_" + fc.name.replace("fp8_", "")
+        try:
+            q, k, v = device_inputs(fc, salt=5)
+            o = torch.empty_like(v)
+            lse = torch.empty((fc.B, fc.H, fc.N), device=dev, dtype=torch.float32)
+            kw = dict(o=o, lse=lse, causal=fc.causal, softmax_scale=fc.softmax_scale, dtype=fa.FA_E4M3_ALL)
+            for _ in range(3):
+                fa.fa_fwd(q, k, v, **kw)
+            times = []
+            for _ in range(5):
+                flush.zero_()
+                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a0.record(stream)
+                fa.fa_fwd(q, k, v, **kw)
+                a1.record(stream)
+                torch.cuda.synchronize()
+                times.append(a0.elapsed_time(a1))
+            ms = statistics.median(times)
+            suite[name] = {"ms": round(ms, 4), "tflops": round(fc.flops / ms / 1e9, 1),
+                           "note": "Q, K, V, P in e4m3; includes the three quantiser passes"}
+            del q, k, v, o, lse
+        except Exception as e:  # report, never hide
+            suite[name] = {"error": str(e)[:200]}
         # ring attention emulated on this GPU (8 sequence blocks, every rank's
         # attention and merge calls in turn, no transfers): the cost of
         # splitting the sequence against the one-launch kernel above

@@ -59,21 +59,29 @@ typedef enum {
 typedef enum {
   FA_BF16 = 0,   /* Q, K, V, O bf16; P rounded to bf16 for the P V product     */
   FA_FP16 = 1,   /* Q, K, V, O fp16; P rounded to fp16                         */
-  FA_E4M3 = 2    /* Q, K given as bf16 and quantised by the library to e4m3
+  FA_E4M3 = 2,   /* Q, K given as bf16 and quantised by the library to e4m3
                     with one scale per (batch, head, 128-row tile); V, O bf16   */
+  FA_E4M3_ALL = 3 /* full FP8: Q, K and V given as bf16 and quantised to e4m3
+                    per (batch, head, 128-row tile); P rounded to e4m3 in the
+                    kernel (scaled by 64 times the ratio of the head's
+                    smallest V scale to the tile's, so that each tile's
+                    product carries the same factor); both products on the
+                    8-bit tensor path.  O bf16.  d = 128.                    */
 } fa_dtype;
 
 /*
  * fa_fwd — the forward pass.
- *   q, k, v : [B, H, N, d] inputs (bf16 / fp16 per dtype; for FA_E4M3, bf16).
+ *   q, k, v : [B, H, N, d] inputs (bf16 / fp16 per dtype; for FA_E4M3 and
+ *             FA_E4M3_ALL, bf16).
  *   o       : [B, H, N, d] output, same element type as v.  Must not alias
  *             q, k or v.
  *   lse     : [B, H, N] fp32 output, or NULL to skip writing it.
  *   softmax_scale : finite, > 0 (typically 1/sqrt(d)).
  *   causal  : 0 or 1.
- * For FA_E4M3 the library quantises q and k into a workspace it owns (grown
- * on demand with cudaMalloc, freed by fa_release) and then runs the FP8
- * attention kernel; this path therefore allocates on first use or growth.
+ * For FA_E4M3 the library quantises q and k (FA_E4M3_ALL: q, k and v) into
+ * a workspace it owns (grown on demand with cudaMalloc, freed by fa_release)
+ * and then runs the FP8 attention kernel; this path therefore allocates on
+ * first use or growth.
  * Returns FA_OK once the work is enqueued.
  */
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,

@@ -1,0 +1,101 @@
+"""GPU parity of the full-FP8 forward (dtype FA_E4M3_ALL: Q, K, V quantised
+to e4m3 per 128-row tile, P rounded to e4m3 in the kernel) against the fp64
+oracle fed the dequantised Q, K and V.
+
+Tolerances.  Against that oracle the one remaining approximation is P: each
+exponential p_j is rounded to e4m3 after scaling by c_j >= 64 * (head's
+smallest V scale / tile's V scale), so its relative error is at most 2^-4
+(3 mantissa bits) in the normal range, and the row sum l is taken from the
+unrounded values.  Hence
+    |O - O_ref| <= sum_j |dp_j| |v_j| / l <= 2^-4 * max_j |v_j|
+up to the subnormal tail (p_j c_j < 2^-6, absolute error <= 2^-10 / c_j),
+which stays far below it on these inputs; the gate is 2^-4 * max|V| plus
+the bf16 half-ulp of the output.  The rounding errors are independent and of
+either sign, so the mean error is much smaller: the mean-abs gate is 2^-4 of
+the mean |O_ref|.  LSE does not see the rounding of P: gated at 1e-3."""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import tiled_attention_12_b200 as fa
+from oracle import attention_ref, attention_rows, dequantize_e4m3_tiles, quantize_e4m3_tiles
+from parity_util import half_ulp, sample_rows
+from tiled_attention_12_b200.synth import WORKLOADS, Case, make_qkv
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _deq(x):
+    c, s = quantize_e4m3_tiles(x)
+    return dequantize_e4m3_tiles(c, s)
+
+
+def _gate(o, lse, ro, rl, vmax, what):
+    o = o.float().cpu().double().numpy()
+    lse = lse.double().cpu().numpy()
+    err = np.abs(o - ro)
+    excess = np.maximum(0.0, err - half_ulp(ro, torch.bfloat16))
+    res = dict(max_excess=float(excess.max()), bound=2.0 ** -4 * vmax, mean=float(err.mean()),
+               mean_bound=2.0 ** -4 * float(np.abs(ro).mean()), lse=float(np.abs(lse - rl).max()))
+    print(what, res)
+    assert np.all(np.isfinite(o)), what
+    assert res["max_excess"] <= res["bound"], (what, res)
+    assert res["mean"] <= res["mean_bound"], (what, res)
+    assert res["lse"] <= 1e-3, (what, res)
+    return res
+
+
+def _run(q, k, v, causal):
+    o, lse = fa.fa_fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=causal, dtype=fa.FA_E4M3_ALL)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status() == 0
+    return o, lse
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [300, 1000, 2048])
+def test_full_fp8_against_dequantised_oracle(N, causal):
+    case = Case("fp8all", 2, 4, N, 128, causal, seed=N + 3)
+    q, k, v = make_qkv(case)
+    o, lse = _run(q, k, v, causal)
+    vd = _deq(v)
+    ro, rl = attention_ref(_deq(q), _deq(k), vd, case.softmax_scale, causal)
+    _gate(o, lse, ro, rl, float(np.abs(vd).max()), f"N{N} c{causal}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_full_fp8_with_outliers(causal):
+    """The FP8 recipe: 1 % of Q, K, V entries times 8."""
+    case = Case("fp8all_out", 1, 4, 2048, 128, causal, seed=7, outlier_frac=0.01, outlier_mult=8.0)
+    q, k, v = make_qkv(case)
+    o, lse = _run(q, k, v, causal)
+    vd = _deq(v)
+    ro, rl = attention_ref(_deq(q), _deq(k), vd, case.softmax_scale, causal)
+    _gate(o, lse, ro, rl, float(np.abs(vd).max()), f"outliers c{causal}")
+
+
+def test_full_fp8_config_shape_sampled_rows():
+    """B2 H16 N16384 d128 causal with 1 % x8 outliers, sampled rows of two heads."""
+    case = WORKLOADS["fp8_b2h16n16384d128_causal"].cases[0]
+    q, k, v = make_qkv(case)
+    o, lse = _run(q, k, v, case.causal)
+    rows = sample_rows(case.N, seed=2, n_random=64)
+    idx = torch.as_tensor(rows, device=DEV)
+    for b, h in ((0, 0), (1, 15)):
+        qd, kd, vd = (_deq(t[b:b + 1, h:h + 1]) for t in (q, k, v))
+        ro, rl = attention_rows(qd, kd, vd, case.softmax_scale, True, 0, 0, rows)
+        _gate(o[b, h][idx], lse[b, h][idx], ro, rl, float(np.abs(vd).max()), f"config ({b},{h})")
+
+
+def test_full_fp8_rejects_other_head_dims_and_block_sparse():
+    q = torch.zeros((1, 1, 256, 64), device=DEV, dtype=torch.bfloat16)
+    with pytest.raises(fa.FaError):
+        fa.fa_fwd(q, q, q.clone(), dtype=fa.FA_E4M3_ALL)
+    q = torch.zeros((1, 1, 256, 128), device=DEV, dtype=torch.bfloat16)
+    mask = torch.ones((1, 1, 2, 2), device=DEV, dtype=torch.uint8)
+    with pytest.raises(fa.FaError):
+        fa.fa_fwd_block_sparse(q, q, q.clone(), mask, dtype=fa.FA_E4M3_ALL)

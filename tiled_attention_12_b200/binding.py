@@ -15,7 +15,7 @@ import re
 from .build import INCLUDE, LIB
 
 FA_OK, FA_ERR_INVALID, FA_ERR_UNSUPPORTED, FA_ERR_ARCH, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_TOO_LARGE = range(7)
-FA_BF16, FA_FP16, FA_E4M3 = 0, 1, 2
+FA_BF16, FA_FP16, FA_E4M3, FA_E4M3_ALL = 0, 1, 2, 3
 
 _lib = None
 
@@ -101,7 +101,8 @@ def fa_fwd(q, k, v, o=None, lse=None, softmax_scale=None, causal=False, dtype=No
     q, k, v may be strided views (for example the (batch, seq, heads, dim)
     layout seen through ``.transpose(1, 2)``) as long as d is contiguous;
     those go through fa_fwd_strided.  dtype: None (from q: bf16 or fp16) or
-    FA_E4M3 (q, k 16-bit, quantised by the library).  Output tensors are
+    FA_E4M3 (q, k 16-bit, quantised by the library) or FA_E4M3_ALL (q, k and
+    v quantised, P rounded to e4m3 in the kernel).  Output tensors are
     allocated when not given (o with v's strides).
     """
     import torch

@@ -130,8 +130,8 @@ bool scale_ok(float s) { return std::isfinite(s) && s > 0.f; }
 // go first; a group's K and V together should stay well inside the 126 MB
 // L2 (about 64 MiB), and groups of at least 4 heads keep the dynamic hand-out
 // balanced at the end of each group.
-int group_heads(int BH, int N, int d, int qk_bytes) {
-  const double kv_head = static_cast<double>(N) * d * (qk_bytes + 2);
+int group_heads(int BH, int N, int d, int qk_bytes, int v_bytes = 2) {
+  const double kv_head = static_cast<double>(N) * d * (qk_bytes + v_bytes);
   int g = static_cast<int>((64.0 * 1024 * 1024) / kv_head);
   if (g < 4) g = 4;
   if (g > 16) g = 16;
@@ -170,24 +170,49 @@ fa_status make_map4(CUtensorMap* map, const void* ptr, int B, int H, int N, int 
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_INVALID;
 }
 
+// e4m3 V codes stored transposed per head, [B, H, d, np] (np = keys padded
+// to a multiple of 128): a 4-D map {N, d, H, B}; box {128 keys, d rows, 1, 1}
+// with the 128-byte swizzle, a K-major tile for the P V product.
+fa_status make_map_vt(CUtensorMap* map, const void* ptr, int B, int H, int N, int d) {
+  const cuuint64_t np = static_cast<cuuint64_t>(fa::transposed_row(N));
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {np, np * d, np * d * H};
+  cuuint32_t box[4] = {128u, static_cast<cuuint32_t>(d), 1u, 1u};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_INVALID;
+}
+
 fa_status launch_attention(DeviceState* ds, int elem, const void* q, const void* k, const void* v, void* o,
                            float* lse, const float* q_scale, const float* k_scale, int B, int H, int N, int d,
                            float softmax_scale, int causal, cudaStream_t stream, const Layout& lay,
-                           const uint16_t* plan = nullptr) {
+                           const uint16_t* plan = nullptr, const float* v_scale = nullptr,
+                           const float* v_scale_min = nullptr) {
   fa::FwdLaunch l;
-  const int qk_bytes = elem == fa::kElemE4M3 ? 1 : 2;
+  const bool all8 = elem == fa::kElemE4M3All;
+  const int qk_bytes = (elem == fa::kElemE4M3 || all8) ? 1 : 2;
+  const int v_bytes = all8 ? 1 : 2;
   const int BH = B * H;
   fa_status st;
   const bool fp16 = elem == fa::kElemF16;
   if ((st = make_map4(&l.map_q, q, B, H, N, d, qk_bytes, fp16, lay.q)) != FA_OK) return st;
   if ((st = make_map4(&l.map_k, k, B, H, N, d, qk_bytes, fp16, lay.k)) != FA_OK) return st;
-  if ((st = make_map4(&l.map_v, v, B, H, N, d, 2, fp16, lay.v)) != FA_OK) return st;
+  if (all8)
+    st = make_map_vt(&l.map_v, v, B, H, N, d);
+  else
+    st = make_map4(&l.map_v, v, B, H, N, d, v_bytes, fp16, lay.v);
+  if (st != FA_OK) return st;
   fa::FwdArgs a;
   std::memset(&a, 0, sizeof(a));
   a.o = o;
   a.lse = lse;
   a.q_scale = q_scale;
   a.k_scale = k_scale;
+  a.v_scale = v_scale;
+  a.v_scale_min = v_scale_min;
   a.status = ds->status;
   a.sched = ds->status + 64 + 2 * (ds->next_slot.fetch_add(1u) % kSchedSlots);
   a.BH = BH;
@@ -208,7 +233,7 @@ fa_status launch_attention(DeviceState* ds, int elem, const void* q, const void*
     g_withhold = 0;
   }
   l.grid = a.n_work < ds->sms ? a.n_work : ds->sms;
-  a.group_heads = group_heads(BH, N, d, qk_bytes);
+  a.group_heads = group_heads(BH, N, d, qk_bytes, v_bytes);
   if (plan != nullptr) {
     a.plan = plan;
     a.plan_stride = fa::block_sparse_plan_stride(N);
@@ -221,6 +246,8 @@ fa_status launch_attention(DeviceState* ds, int elem, const void* q, const void*
     e = fa::launch_fwd_bf16(d, l);
   else if (elem == fa::kElemF16)
     e = fa::launch_fwd_f16(d, l);
+  else if (all8)
+    e = fa::launch_fwd_e4m3_all(d, l);
   else
     e = fa::launch_fwd_e4m3(d, l);
   return map_cuda(e);
@@ -232,36 +259,56 @@ struct Quantised {
   uint8_t* k8;
   float* qs;
   float* ks;
+  uint8_t* v8 = nullptr;     // FA_E4M3_ALL only
+  float* vs = nullptr;
+  float* vs_min = nullptr;   // [B*H]
 };
 
+// v != nullptr: quantise v as well (FA_E4M3_ALL) and find each head's
+// smallest V tile scale.
 fa_status quantise_qk(DeviceState* ds, const void* q, const void* k, int B, int H, int N, int d, const Layout& lay,
-                      cudaStream_t s, Quantised* out) {
+                      cudaStream_t s, Quantised* out, const void* v = nullptr) {
   const int BH = B * H;
   const size_t elems = static_cast<size_t>(BH) * N * d;
   const size_t n_scales = static_cast<size_t>(BH) * ((N + 127) / 128);
   const size_t codes_bytes = (elems + 255) & ~static_cast<size_t>(255);
-  const size_t need = 2 * codes_bytes + 2 * n_scales * sizeof(float);
+  const size_t scales_bytes = (n_scales * sizeof(float) + 255) & ~static_cast<size_t>(255);
+  // transposed V codes: [BH, d, keys padded to 128]
+  const size_t vt_bytes = v ? ((static_cast<size_t>(BH) * d * fa::transposed_row(N) + 255) & ~static_cast<size_t>(255))
+                            : 0;
+  const size_t n_ops = v ? 3 : 2;
+  const size_t need = 2 * codes_bytes + vt_bytes + n_ops * scales_bytes +
+                      (v ? static_cast<size_t>(BH) * sizeof(float) : 0);
   {
     std::lock_guard<std::mutex> lock(g_mu);
     fa_status st = grow(&ds->ws, &ds->ws_bytes, need);
     if (st != FA_OK) return st;
   }
-  out->q8 = static_cast<uint8_t*>(ds->ws);
-  out->k8 = out->q8 + codes_bytes;
-  out->qs = reinterpret_cast<float*>(out->k8 + codes_bytes);
-  out->ks = out->qs + n_scales;
+  uint8_t* base = static_cast<uint8_t*>(ds->ws);
+  out->q8 = base;
+  out->k8 = base + codes_bytes;
+  uint8_t* sc = base + 2 * codes_bytes + vt_bytes;
+  out->qs = reinterpret_cast<float*>(sc);
+  out->ks = reinterpret_cast<float*>(sc + scales_bytes);
   if (fa::launch_quantize_e4m3(q, out->q8, out->qs, B, H, N, d, lay.q, s) != cudaSuccess) return FA_ERR_CUDA;
   if (fa::launch_quantize_e4m3(k, out->k8, out->ks, B, H, N, d, lay.k, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (v != nullptr) {
+    out->v8 = base + 2 * codes_bytes;
+    out->vs = reinterpret_cast<float*>(sc + 2 * scales_bytes);
+    out->vs_min = reinterpret_cast<float*>(sc + 3 * scales_bytes);
+    if (fa::launch_quantize_e4m3_t(v, out->v8, out->vs, B, H, N, d, lay.v, s) != cudaSuccess) return FA_ERR_CUDA;
+    if (fa::launch_min_scale(out->vs, out->vs_min, BH, N, s) != cudaSuccess) return FA_ERR_CUDA;
+  }
   return FA_OK;
 }
 
 // Checks shared by the forward entry points (before any CUDA call).
 fa_status check_forward(const void* q, const void* k, const void* v, void* o, const float* lse, int B, int H, int N,
                         int d, float softmax_scale, int causal, fa_dtype dtype) {
-  if (dtype != FA_BF16 && dtype != FA_FP16 && dtype != FA_E4M3) return FA_ERR_INVALID;
+  if (dtype != FA_BF16 && dtype != FA_FP16 && dtype != FA_E4M3 && dtype != FA_E4M3_ALL) return FA_ERR_INVALID;
   fa_status st = check_shape(B, H, N, d);
   if (st != FA_OK) return st;
-  if (dtype == FA_E4M3 && d != 128) return FA_ERR_UNSUPPORTED;
+  if ((dtype == FA_E4M3 || dtype == FA_E4M3_ALL) && d != 128) return FA_ERR_UNSUPPORTED;
   if (!q || !k || !v || !o) return FA_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)))
     return FA_ERR_INVALID;
@@ -291,8 +338,14 @@ fa_status forward(const void* q, const void* k, const void* v, void* o, float* l
     return launch_attention(ds, dtype == FA_BF16 ? fa::kElemBF16 : fa::kElemF16, q, k, v, o, lse, nullptr, nullptr, B,
                             H, N, d, softmax_scale, causal, s, lay, plan);
   Quantised qz;
-  if ((st = quantise_qk(ds, q, k, B, H, N, d, lay, s, &qz)) != FA_OK) return st;
+  const bool all8 = dtype == FA_E4M3_ALL;
+  if ((st = quantise_qk(ds, q, k, B, H, N, d, lay, s, &qz, all8 ? v : nullptr)) != FA_OK) return st;
   const fa::Strides codes = fa::contiguous_strides(H, N, d);
+  if (all8) {
+    const Layout lay8{codes, codes, codes, lay.o};
+    return launch_attention(ds, fa::kElemE4M3All, qz.q8, qz.k8, qz.v8, o, lse, qz.qs, qz.ks, B, H, N, d, softmax_scale,
+                            causal, s, lay8, plan, qz.vs, qz.vs_min);
+  }
   const Layout lay8{codes, codes, lay.v, lay.o};
   return launch_attention(ds, fa::kElemE4M3, qz.q8, qz.k8, v, o, lse, qz.qs, qz.ks, B, H, N, d, softmax_scale, causal,
                           s, lay8, plan);
@@ -339,7 +392,7 @@ fa_status fa_fwd_block_sparse(const void* q, const void* k, const void* v, void*
                               void* stream) {
   fa_status st = check_forward(q, k, v, o, lse, B, H, N, d, softmax_scale, causal, dtype);
   if (st != FA_OK) return st;
-  if ((N + 127) / 128 > fa::kPlanMaxTiles) return FA_ERR_UNSUPPORTED;
+  if ((N + 127) / 128 > fa::kPlanMaxTiles || dtype == FA_E4M3_ALL) return FA_ERR_UNSUPPORTED;
   if (!block_mask) return FA_ERR_INVALID;
   return forward(q, k, v, o, lse, B, H, N, d, softmax_scale, causal, dtype, static_cast<cudaStream_t>(stream),
                  contiguous_layout(H, N, d), block_mask);

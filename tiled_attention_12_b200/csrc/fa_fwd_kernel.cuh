@@ -61,7 +61,9 @@
 
 namespace fa {
 
-enum : int { kElemBF16 = 0, kElemF16 = 1, kElemE4M3 = 2 };
+// kElemE4M3: e4m3 Q, K (per-tile scales), bf16 V and P.  kElemE4M3All: V
+// and P in e4m3 too, so both products run at the 8-bit tensor rate.
+enum : int { kElemBF16 = 0, kElemF16 = 1, kElemE4M3 = 2, kElemE4M3All = 3 };
 
 // Status bits written to the device status word when a wait gives up.
 enum : unsigned { kStatusProducer = 1u, kStatusMma = 2u, kStatusSoftmax = 4u, kStatusDrain = 8u };
@@ -82,6 +84,8 @@ struct FwdArgs {
   float* lse;              // [BH, N] fp32 or nullptr
   const float* q_scale;    // [BH, ceil(N/128)] (e4m3 only)
   const float* k_scale;    // [BH, ceil(N/128)] (e4m3 only)
+  const float* v_scale;    // [BH, ceil(N/128)] (e4m3 V only)
+  const float* v_scale_min;  // [BH]: smallest V tile scale of the head (e4m3 V only)
   unsigned int* status;    // device status word
   unsigned int* sched;     // this launch's scheduler counters: [0] next work tile, [1] CTAs done
   int BH;                  // batch * heads
@@ -112,9 +116,12 @@ template <int D, int ELEM>
 struct FwdCfg {
   static constexpr int BM = 128;  // query rows per Q tile = MMA M
   static constexpr int BN = 128;  // keys per K/V tile = S MMA N
-  static constexpr int QK_BYTES = (ELEM == kElemE4M3) ? 1 : 2;
+  static constexpr bool QK8 = ELEM == kElemE4M3 || ELEM == kElemE4M3All;  // e4m3 Q, K
+  static constexpr bool PV8 = ELEM == kElemE4M3All;                        // e4m3 P, V
+  static constexpr int QK_BYTES = QK8 ? 1 : 2;
+  static constexpr int V_BYTES = PV8 ? 1 : 2;
   static constexpr int QK_ROW = D * QK_BYTES;
-  static constexpr int V_ROW = D * 2;
+  static constexpr int V_ROW = D * V_BYTES;
   static constexpr int SW_QK = QK_ROW >= 128 ? 128 : QK_ROW;  // swizzle span in bytes
   static constexpr int SW_V = V_ROW >= 128 ? 128 : V_ROW;
   static_assert(SW_QK == 128 || SW_QK == 64, "head dim gives an unsupported swizzle span");
@@ -135,7 +142,8 @@ struct FwdCfg {
   static constexpr int SMEM_BYTES = SMEM_NEED > 120 * 1024 ? SMEM_NEED : 120 * 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget exceeded");
   static constexpr int K_STEPS_QK = QK_ROW / 32;   // 32 bytes of K per S MMA (16 x 16-bit or 32 x 8-bit)
-  static constexpr int K_STEPS_PV = BN / 16;       // 16 keys per P V MMA
+  static constexpr int PV_K = PV8 ? 32 : 16;      // keys per P V MMA (32 bytes of P per row either way)
+  static constexpr int K_STEPS_PV = BN / PV_K;
   static constexpr int THREADS = 384;  // 3 warpgroups
   static constexpr int MMA_WARP = 8;    // MMA issuer (Q tile 0 when decoupled); allocates tensor memory
   static constexpr int LOAD_WARP = 9;
@@ -162,11 +170,18 @@ struct FwdCfg {
   static_assert(O_COL1 + D <= TMEM_COLS, "tensor memory budget exceeded");
   static constexpr uint32_t IDESC_QK =
       instr_desc(ELEM == kElemBF16 ? 1u : 0u, ELEM == kElemBF16 ? 1u : 0u, 0u, BM, BN);
-  static constexpr uint32_t IDESC_PV =
-      instr_desc(ELEM == kElemF16 ? 0u : 1u, ELEM == kElemF16 ? 0u : 1u, 1u, BM, D);
+  // e4m3 V is stored transposed ([d, keys] per head), so its tile is a
+  // K-major operand like K's; 16-bit V is read MN-major.
+  static constexpr uint32_t IDESC_PV = PV8 ? instr_desc(0u, 0u, 0u, BM, D)
+                                          : instr_desc(ELEM == kElemF16 ? 0u : 1u, ELEM == kElemF16 ? 0u : 1u, 1u, BM, D);
   static constexpr uint32_t SWZ_QK = SW_QK == 128 ? 2u : 4u;
   static constexpr uint32_t SWZ_V = SW_V == 128 ? 2u : 4u;
-  static constexpr float TAU = 8.0f;  // deferred-rescale threshold (log2 units)
+  // Deferred-rescale threshold (log2 units): p <= 2^TAU.  With e4m3 P the
+  // exponentials are scaled by 2^P_SCALE_LOG2 (times the V tile factor <= 1)
+  // before rounding, so that small p keep precision, and the bound
+  // 2^(TAU + P_SCALE_LOG2) = 256 stays below e4m3's largest value, 448.
+  static constexpr float TAU = PV8 ? 2.0f : 8.0f;
+  static constexpr float P_SCALE_LOG2 = PV8 ? 6.0f : 0.0f;
   // Column pairs (of every 16) whose exponentials use the FMA-pipe
   // polynomial instead of the special-function unit: 5 of 16 pairs.
   static constexpr uint32_t POLY_MASK = FA_POLY_MASK;
@@ -452,9 +467,15 @@ __device__ __forceinline__ void producer_role(const FwdArgs& a, const Bars<FwdCf
                         th, tb);
         } else {
           mbar_arrive_expect_tx(b.kv_full(s), C::V_TILE);
+          if constexpr (C::PV8) {
+            // transposed codes: one box of 128 keys x D rows
+            tma_load_4d(dst, map_v, b.kv_full(s), j * 128, 0, th, tb);
+          } else {
 #pragma unroll
-          for (int c = 0; c < C::V_ROW / C::SW_V; ++c)
-            tma_load_4d(dst + c * C::BN * C::SW_V, map_v, b.kv_full(s), c * (C::SW_V / 2), j * 128, th, tb);
+            for (int c = 0; c < C::V_ROW / C::SW_V; ++c)
+              tma_load_4d(dst + c * C::BN * C::SW_V, map_v, b.kv_full(s), c * (C::SW_V / C::V_BYTES), j * 128, th,
+                          tb);
+          }
         }
       }
     }
@@ -486,7 +507,8 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const Bars<FwdCfg<D, 
   const uint64_t limit = a.wait_limit_ns;
   const uint64_t dq0 = smem_desc(sQ_addr, 16, 8 * C::SW_QK, C::SWZ_QK);
   const uint64_t dkv0 = smem_desc(sKV_addr, 16, 8 * C::SW_QK, C::SWZ_QK);
-  const uint64_t dv0 = smem_desc(sKV_addr, C::BN * C::SW_V, 8 * C::SW_V, C::SWZ_V);
+  const uint64_t dv0 = C::PV8 ? smem_desc(sKV_addr, 16, 8 * 128, 2u)  // [D rows][128 keys], 128-byte swizzle
+                             : smem_desc(sKV_addr, C::BN * C::SW_V, 8 * C::SW_V, C::SWZ_V);
   int kv_it = 0, q_use0 = 0, q_use1 = 0, p_cnt0 = 0, p_cnt1 = 0;
   FA_TRACE_DECL;
 
@@ -497,7 +519,7 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const Bars<FwdCfg<D, 
 #pragma unroll
     for (int kk = 0; kk < C::K_STEPS_QK; ++kk) {
       const uint32_t off = ((kk * 32) / C::SW_QK) * (C::BM * C::SW_QK) + ((kk * 32) % C::SW_QK);
-      if constexpr (ELEM == kElemE4M3)
+      if constexpr (C::QK8)
         mma_f8_ss(d_tmem, qa + (off >> 4), ka + (off >> 4), C::IDESC_QK, kk > 0);
       else
         mma_f16_ss(d_tmem, qa + (off >> 4), ka + (off >> 4), C::IDESC_QK, kk > 0);
@@ -511,8 +533,13 @@ __device__ __forceinline__ void mma_role(const FwdArgs& a, const Bars<FwdCfg<D, 
 #pragma unroll
     for (int k = 0; k < C::K_STEPS_PV / 2; ++k) {
       const int kk = half * (C::K_STEPS_PV / 2) + k;
-      mma_f16_ts(d_tmem, p_tmem + kk * 8, va + ((kk * 16 * C::SW_V) >> 4), C::IDESC_PV,
-                 (accumulate || kk > 0) ? 1u : 0u);
+      // 16-bit V: PV_K rows of the [keys, D] tile per MMA; e4m3 V: 32 bytes
+      // (32 keys) along each row of the [D, keys] tile
+      const uint64_t vb = va + (C::PV8 ? ((kk * 32) >> 4) : ((kk * C::PV_K * C::SW_V) >> 4));
+      if constexpr (C::PV8)
+        mma_f8_ts(d_tmem, p_tmem + kk * 8, vb, C::IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
+      else
+        mma_f16_ts(d_tmem, p_tmem + kk * 8, vb, C::IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
     }
   };
   // P_i arrives in two halves, each on its own barrier (one phase per step),
@@ -774,6 +801,43 @@ __device__ __forceinline__ void exp_store_half(const uint32_t (&sr)[4][32], int 
   }
 }
 
+// exp_store_half for e4m3 P: the 64 exponentials of `half` (already scaled
+// by the caller's exponent offset) rounded to e4m3, four per tensor-memory
+// column (lowest key in the lowest byte), 16 columns at t_p + 16 * half.
+template <uint32_t POLY_MASK>
+__device__ __forceinline__ void exp_store_half_e4m3(const uint32_t (&sr)[4][32], int half, uint64_t sl2x2,
+                                                    uint64_t negm2, uint32_t t_p, uint64_t& acc_a, uint64_t& acc_b) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int cc = 0; cc < 2; ++cc) {
+    const int c = 2 * half + cc;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const uint64_t x2 = ffma2(pack2(FA_S(c * 32 + 2 * e), FA_S(c * 32 + 2 * e + 1)), sl2x2, negm2);
+      uint64_t p2;
+      if ((POLY_MASK >> e) & 1u) {
+        p2 = exp2_poly2(x2);
+      } else {
+        float x0, x1;
+        unpack2(x2, x0, x1);
+        p2 = pack2(ex2_approx(x0), ex2_approx(x1));
+      }
+      if (e & 1)
+        acc_b = fadd2(acc_b, p2);
+      else
+        acc_a = fadd2(acc_a, p2);
+      float p0, p1;
+      unpack2(p2, p0, p1);
+      const uint32_t two = cvt_e4m3x2(p0, p1);
+      if (e & 1)
+        pk[cc * 8 + (e >> 1)] |= two << 16;
+      else
+        pk[cc * 8 + (e >> 1)] = two;
+    }
+  }
+  tmem_st16(t_p + half * 16, pk);
+}
+
 // Same as exp_store_half for all 128 columns, but the packed P stays in
 // registers (pk[chunk][16]) so it can be stored later.
 template <int ELEM, uint32_t POLY_MASK>
@@ -816,10 +880,12 @@ __device__ __forceinline__ float sum_acc(uint64_t acc_a, uint64_t acc_b) {
 }
 
 // O / l of this thread's row to global memory (16-byte stores), and LSE.
+// o_scale: undoes a scale the P V products carried (1 unless P and V are e4m3).
 template <int D, int ELEM>
-__device__ __forceinline__ void epilogue_row(const FwdArgs& a, uint32_t t_o, int bh, int qrow, float m, float l) {
+__device__ __forceinline__ void epilogue_row(const FwdArgs& a, uint32_t t_o, int bh, int qrow, float m, float l,
+                                             float o_scale = 1.f) {
   using OutT = typename std::conditional<ELEM == kElemF16, __half, __nv_bfloat16>::type;
-  const float inv_l = 1.f / l;
+  const float inv_l = o_scale / l;
   OutT* orow = o_row<OutT>(a, bh, qrow);
 #pragma unroll
   for (int c = 0; c < D / 32; ++c) {
@@ -904,7 +970,12 @@ __device__ __forceinline__ void softmax_role(const FwdArgs& a, const Bars<FwdCfg
         continue;
       }
       float sl2_q = a.scale_log2;
-      if constexpr (ELEM == kElemE4M3) sl2_q = a.scale_log2 / a.q_scale[t.bh * a.n_qtiles + (q_start >> 7)];
+      if constexpr (C::QK8) sl2_q = a.scale_log2 / a.q_scale[t.bh * a.n_qtiles + (q_start >> 7)];
+      // e4m3 V: tile j's codes carry scale v_scale[j]; P is scaled by
+      // 2^P_SCALE_LOG2 * vmin / v_scale[j] so that every tile's P V product
+      // carries the same factor 2^P_SCALE_LOG2 * vmin, undone in the epilogue
+      float vmin = 1.f;
+      if constexpr (C::PV8) vmin = a.v_scale_min[t.bh];
       float m = -INFINITY;  // running max, log2 units of the scaled score
       float l = 0.f;        // running sum of exponentials
       for (int step = 0; step < nkv; ++step) {
@@ -915,7 +986,9 @@ __device__ __forceinline__ void softmax_role(const FwdArgs& a, const Bars<FwdCfg
         tc_fence_after();
         if (lane == 0 && wq == 0) FA_TRACE_EV(wg, 1 + 10 * wg, j);
         float sl2 = sl2_q;
-        if constexpr (ELEM == kElemE4M3) sl2 = sl2_q / a.k_scale[t.bh * a.n_qtiles + j];
+        if constexpr (C::QK8) sl2 = sl2_q / a.k_scale[t.bh * a.n_qtiles + j];
+        float lc = 0.f;  // log2 of the factor on this tile's exponentials
+        if constexpr (C::PV8) lc = C::P_SCALE_LOG2 + __log2f(vmin / a.v_scale[t.bh * a.n_qtiles + j]);
         uint32_t sr[4][32];
         load_s_row(t_s, sr);
         if (BS ? tile_needs_mask(a, j, q_start) : step == nkv - 1) mask_row(sr, j * 128, (a.causal && qrow < a.N - 1) ? qrow : a.N - 1);
@@ -931,11 +1004,14 @@ __device__ __forceinline__ void softmax_role(const FwdArgs& a, const Bars<FwdCfg
           rescale_o<D>(t_o, alpha);
         }
         const uint64_t sl2x2 = pack2(sl2, sl2);
-        const uint64_t negm2 = pack2(-m, -m);
+        const uint64_t negm2 = pack2(lc - m, lc - m);
         uint64_t acc_a = pack2(0.f, 0.f), acc_b = pack2(0.f, 0.f);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          exp_store_half<ELEM, C::POLY_MASK>(sr, half, sl2x2, negm2, t_s, acc_a, acc_b);
+          if constexpr (C::PV8)
+            exp_store_half_e4m3<C::POLY_MASK>(sr, half, sl2x2, negm2, t_s, acc_a, acc_b);
+          else
+            exp_store_half<ELEM, C::POLY_MASK>(sr, half, sl2x2, negm2, t_s, acc_a, acc_b);
           if (FA_SPLIT_P || half == 1) {
             tmem_st_wait();
             tc_fence_before();
@@ -944,14 +1020,20 @@ __device__ __forceinline__ void softmax_role(const FwdArgs& a, const Bars<FwdCfg
             if (lane == 0 && wq == 0) FA_TRACE_EV(wg, 3 + half + 10 * wg, j);
           }
         }
-        l += sum_acc(acc_a, acc_b);
+        if constexpr (C::PV8)
+          l += sum_acc(acc_a, acc_b) * ex2_approx(-lc);
+        else
+          l += sum_acc(acc_a, acc_b);
       }
       feed_release_warp<BS>(feed, slot, lane);
       // epilogue: O / l -> global, LSE
       if (!wait_warp(o_full, o_cnt)) return false;
       ++o_cnt;
       tc_fence_after();
-      epilogue_row<D, ELEM>(a, t_o, t.bh, qrow, m, l);
+      if constexpr (C::PV8)
+        epilogue_row<D, ELEM>(a, t_o, t.bh, qrow, m, l, ex2_approx(-C::P_SCALE_LOG2) / vmin);
+      else
+        epilogue_row<D, ELEM>(a, t_o, t.bh, qrow, m, l);
     }
     return true;
   };
@@ -1082,7 +1164,7 @@ __device__ __forceinline__ void mma_role_decoupled(const FwdArgs& a, const Bars<
                                                    uint32_t sQ_addr, uint32_t sKV_addr, uint32_t tmem,
                                                    const TileFeed feed, volatile int* abort_flag) {
   using C = FwdCfg<D, ELEM>;
-  static_assert(ELEM != kElemE4M3, "the e4m3 path uses the aliased layout");
+  static_assert(!C::QK8, "the e4m3 paths use the aliased layout");
   const uint64_t limit = a.wait_limit_ns;
   const uint64_t dq = smem_desc(sQ_addr + i * C::Q_TILE, 16, 8 * C::SW_QK, C::SWZ_QK);
   const uint64_t dkv0 = smem_desc(sKV_addr, 16, 8 * C::SW_QK, C::SWZ_QK);

@@ -37,6 +37,14 @@ cudaError_t launch_fwd_sparse(int d, int elem, const FwdLaunch& l);
 // 16-bit input read at strides `st`.
 cudaError_t launch_quantize_e4m3(const void* x, void* x8, float* scales, int B, int H, int N, int d,
                                  const Strides& st, cudaStream_t stream);
+// The same codes written transposed per head, [B*H, d, transposed_row(N)]
+// (keys contiguous, padded to a multiple of 128 with zeros), same scales.
+long long transposed_row(int N);
+cudaError_t launch_quantize_e4m3_t(const void* x, void* x8t, float* scales, int B, int H, int N, int d,
+                                   const Strides& st, cudaStream_t stream);
+// Per head, the smallest of its per-tile scales ([BH, ceil(N/128)] -> [BH]).
+cudaError_t launch_min_scale(const float* scales, float* out, int BH, int N, cudaStream_t stream);
+cudaError_t launch_fwd_e4m3_all(int d, const FwdLaunch& l);
 int fwd_smem_bytes(int d, int elem);
 // Block-sparse plan rows (layout in fa_fwd_kernel.cuh) from a uint8 block
 // mask [BH, ceil(N/128), ceil(N/128)].
