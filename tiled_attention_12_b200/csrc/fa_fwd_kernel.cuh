@@ -47,8 +47,13 @@
 
 #include "ptx.cuh"
 
-#ifndef FA_POLY_MASK
-#define FA_POLY_MASK 0x4924u
+// Column pairs (bit e of every 16) whose exponentials use the FMA-pipe
+// polynomial instead of the special-function unit, per head dimension.
+#ifndef FA_POLY_MASK_SMALL
+#define FA_POLY_MASK_SMALL 0x4924u  // d <= 64: 5 of 16 pairs
+#endif
+#ifndef FA_POLY_MASK_D128
+#define FA_POLY_MASK_D128 0x0000u   // d = 128: none
 #endif
 // 1: the softmax hands P to the MMA warp in two halves (keys 0-63, 64-127)
 #ifndef FA_SPLIT_P
@@ -182,9 +187,11 @@ struct FwdCfg {
   // 2^(TAU + P_SCALE_LOG2) = 256 stays below e4m3's largest value, 448.
   static constexpr float TAU = PV8 ? 2.0f : 8.0f;
   static constexpr float P_SCALE_LOG2 = PV8 ? 6.0f : 0.0f;
-  // Column pairs (of every 16) whose exponentials use the FMA-pipe
-  // polynomial instead of the special-function unit: 5 of 16 pairs.
-  static constexpr uint32_t POLY_MASK = FA_POLY_MASK;
+  // Measured by interleaved A/B on B200: at d <= 64 the exponentials bound
+  // the kernel and moving 5 of 16 pairs to the FMA pipe is fastest; at
+  // d = 128 the softmax shares the SM with twice the tensor work per score
+  // and the polynomial's extra instructions cost more than they save.
+  static constexpr uint32_t POLY_MASK = D >= 128 ? FA_POLY_MASK_D128 : FA_POLY_MASK_SMALL;
 };
 
 // Barrier slots (8 bytes each) after the tiles in shared memory, addressed by
