@@ -206,6 +206,8 @@ __global__ void __launch_bounds__(320, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t tmem_holder;
   __shared__ int abort_storage;
+  // per compute warp: LSE (log2 units) and D of its 64 query columns
+  __shared__ __align__(16) float lse_d_stage[8][2][64];
   volatile int* abort_flag = &abort_storage;
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sK = (raw + 1023u) & ~1023u;
@@ -310,9 +312,34 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t tS = tmem + lane_off + C::COL_A, tP = tmem + lane_off + C::COL_B;
     const float* lse_h = a.lse + static_cast<size_t>(bh) * a.N;
     const float* dlt_h = a.delta + static_cast<size_t>(bh) * a.N;
+    // LSE and D of this warp's 64 query columns, fetched one query block
+    // ahead: lane l holds columns l and 32 + l in registers, and at the top of
+    // each block the warp publishes them in its own shared-memory slot (only
+    // __syncwarp orders it), from which every lane reads them as broadcasts.
+    float pre_l[2], pre_d[2];
+    auto prefetch = [&](int tt) {
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int qq = (i0 + tt) * 128 + 64 * half + 32 * u + lane;
+        const bool in_seq = tt < n_i && qq < a.N;
+        pre_l[u] = in_seq ? lse_h[qq] * 1.4426950408889634f : 0.f;
+        pre_d[u] = in_seq ? dlt_h[qq] : 0.f;
+      }
+    };
+    prefetch(0);
+    float* stage_l = lse_d_stage[warp][0];
+    float* stage_d = lse_d_stage[warp][1];
     bool ok = true;
     for (int t = 0; t < n_i && ok; ++t) {
       const int qb = (i0 + t) * 128;
+      __syncwarp();  // every lane is done reading the previous block's values
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        stage_l[32 * u + lane] = pre_l[u];
+        stage_d[32 * u + lane] = pre_d[u];
+      }
+      __syncwarp();
+      prefetch(t + 1);  // in flight while this block computes
       ok = __all_sync(0xffffffffu, wait_bounded(b.s_full(), t & 1, abort_flag, limit));
       if (!ok) break;
       tc_fence_after();
@@ -321,23 +348,16 @@ __global__ void __launch_bounds__(320, 1)
         ChunkIn in;
         tmem_ld32(tS + 32 * c, in.s);
         tmem_ld32(tP + 32 * c, in.dp);
-        // LSE and D of the chunk's 32 queries (the same for every lane)
+        // LSE (log2 units) and D of the chunk's 32 queries (the same for every lane)
         const int q0 = qb + 32 * c;
         float lse2[32], dlt[32];
-        if (q0 + 32 <= a.N && ((reinterpret_cast<uintptr_t>(lse_h + q0) | reinterpret_cast<uintptr_t>(dlt_h + q0)) & 15) == 0) {
+        const float4* sl4 = reinterpret_cast<const float4*>(stage_l + 32 * (c - 2 * half));
+        const float4* sd4 = reinterpret_cast<const float4*>(stage_d + 32 * (c - 2 * half));
 #pragma unroll
-          for (int v4 = 0; v4 < 8; ++v4) {
-            const float4 l4 = reinterpret_cast<const float4*>(lse_h + q0)[v4];
-            const float4 d4 = reinterpret_cast<const float4*>(dlt_h + q0)[v4];
-            lse2[4 * v4] = l4.x; lse2[4 * v4 + 1] = l4.y; lse2[4 * v4 + 2] = l4.z; lse2[4 * v4 + 3] = l4.w;
-            dlt[4 * v4] = d4.x; dlt[4 * v4 + 1] = d4.y; dlt[4 * v4 + 2] = d4.z; dlt[4 * v4 + 3] = d4.w;
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            lse2[e] = q0 + e < a.N ? lse_h[q0 + e] : 0.f;
-            dlt[e] = q0 + e < a.N ? dlt_h[q0 + e] : 0.f;
-          }
+        for (int v4 = 0; v4 < 8; ++v4) {
+          const float4 l4 = sl4[v4], d4 = sd4[v4];
+          lse2[4 * v4] = l4.x; lse2[4 * v4 + 1] = l4.y; lse2[4 * v4 + 2] = l4.z; lse2[4 * v4 + 3] = l4.w;
+          dlt[4 * v4] = d4.x; dlt[4 * v4 + 1] = d4.y; dlt[4 * v4 + 2] = d4.z; dlt[4 * v4 + 3] = d4.w;
         }
         tmem_ld_wait(in.s);
         reg_tie(in.dp);
@@ -349,7 +369,7 @@ __global__ void __launch_bounds__(320, 1)
           for (int u = 0; u < 2; ++u) {
             const int qq = q0 + e + u;
             const bool valid = qq < a.N && !(a.causal && qq < key);
-            const float p = ex2_approx(fmaf(__uint_as_float(in.s[e + u]), a.scale_log2, -lse2[e + u] * 1.4426950408889634f));
+            const float p = ex2_approx(fmaf(__uint_as_float(in.s[e + u]), a.scale_log2, -lse2[e + u]));
             pv[u] = valid ? p : 0.f;
             dv[u] = pv[u] * (__uint_as_float(in.dp[e + u]) - dlt[e + u]);
           }
