@@ -17,12 +17,17 @@
 //              O rescale, epilogue (O / l, LSE)
 //   warps 4-7  softmax warpgroup 1 (Q tile 1)
 //   warp  8    MMA issuer (one thread): S_i = Q_i K^T and O_i += P_i V on the
-//              tensor cores, accumulators in tensor memory
-//   warp  9    TMA producer (one thread): Q tiles and a ring of K/V tiles
+//              tensor cores, accumulators in tensor memory (d <= 64: warp 10
+//              issues Q tile 1's products)
+//   warp  9    TMA producer (one thread): Q tiles and a ring of K/V tiles,
+//              through 4-D tensor maps {d, N, H, B} built from the caller's
+//              strides
 //
-// Tensor memory (512 fp32 columns x 128 lanes, lane = query row):
+// Tensor memory at d = 128 (512 fp32 columns x 128 lanes, lane = query row):
 //   S_0 [0,128)  S_1 [128,256)  O_0 [256,256+D)  O_1 [256+D,256+2D)
-//   P_i (16-bit) overwrites the first 64 columns of S_i once S_i is read.
+//   P_i overwrites the first 64 columns of S_i (16-bit P) or the first 32
+//   (e4m3 P) once S_i is read.  At d <= 64 P has columns of its own (see
+//   FwdCfg: DECOUPLED).
 //
 // MMA order per K/V step j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1).  While one
 // warpgroup exponentiates its scores, the tensor cores run the other Q tile's
