@@ -342,6 +342,31 @@ def run_ours(args, rank, world, local_rank):
                     del q, k, v, o, lse
                 except Exception as e:  # report, never hide
                     suite[c.name] = {"error": str(e)[:200]}
+        # the small cases of the default workload with and without an L2 flush
+        # between launches (back to back, inputs warm in L2)
+        for c in [c for c in WORKLOADS["dmodel512_h16"].cases if c.N <= 1024]:
+            name = c.name + "_l2warm"
+            try:
+                q, k, v = device_inputs(c, salt=6)
+                o = torch.empty_like(v)
+                lse = torch.empty((c.B, c.H, c.N), device=dev, dtype=torch.float32)
+                kw = dict(o=o, lse=lse, causal=c.causal, softmax_scale=c.softmax_scale)
+                for _ in range(10):
+                    fa.fa_fwd(q, k, v, **kw)
+                times = []
+                for _ in range(50):
+                    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a0.record(stream)
+                    fa.fa_fwd(q, k, v, **kw)
+                    a1.record(stream)
+                    torch.cuda.synchronize()
+                    times.append(a0.elapsed_time(a1))
+                ms = statistics.median(times)
+                suite[name] = {"ms": round(ms, 4), "ms_min": round(min(times), 4),
+                               "tflops": round(c.flops / ms / 1e9, 1), "note": "no L2 flush between launches"}
+                del q, k, v, o, lse
+            except Exception as e:  # report, never hide
+                suite[name] = {"error": str(e)[:200]}
         # backward (fa_bwd) on the d=128 shapes: algorithmic FLOPs 2.5x the
         # forward's (five N x N x d products: S, dP, dV, dK, dQ)
         for c in list(WORKLOADS["target_d128_noncausal"].cases[:1]) + list(WORKLOADS["b4h16n8192d128_causal"].cases):

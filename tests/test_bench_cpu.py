@@ -1,0 +1,56 @@
+"""bench.py on the CPU: the reference arm's JSON line follows the contract,
+and the helpers the GPU arm uses agree with the oracle's accounting."""
+
+from __future__ import annotations
+
+import importlib.util
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench_module():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_reference_arm_json_line():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "0"], capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "TFLOPS"
+    assert line["higher_is_better"] is True and line["n_gpus"] == 1 and line["steps"] == 1
+    assert line["config"]["workload"] == "dmodel512_h16"
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["e2e"]["value"] == line["value"]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1000, 8192])
+def test_block_sparse_flops_match_oracle_count(N, causal):
+    from oracle.block_sparse import block_sparse_flops
+    from tiled_attention_12_b200.synth import make_block_mask
+
+    bench = _bench_module()
+    for kind in ("random", "window", "ones"):
+        m = make_block_mask(2, 3, N, kind, 0.5, window=3, seed=1)
+        assert bench.block_sparse_pair_count(m, N, causal) * 4 * 64 == block_sparse_flops(m, N, 64, causal)
+
+
+def test_kernel_source_hash_covers_the_forward_sources():
+    bench = _bench_module()
+    h = bench.kernel_source_hash()
+    assert isinstance(h, str) and len(h) == 16 and h == bench.kernel_source_hash()
