@@ -70,30 +70,32 @@ struct BwdCfg {
   static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
   static_assert(NS >= 2, "ring too shallow");
   static constexpr int BYTES = FIXED + NS * STAGE;
-  static constexpr int NUM_BARS = 2 * NS + 5;
+  static constexpr int NUM_BARS = 2 * NS + 7;
   static constexpr int SMEM_NEED = 1024 + BYTES + 8 * NUM_BARS;
   static constexpr int SMEM_BYTES = SMEM_NEED > 120 * 1024 ? SMEM_NEED : 120 * 1024;  // one CTA per SM
   static_assert(SMEM_BYTES <= 232448, "shared memory budget exceeded");
   static constexpr int K_STEPS = ROW / 32;                    // 16 elements per MMA K step
   static constexpr uint32_t FMT = ELEM == 1 ? 0u : 1u;        // f16 : bf16
   static constexpr uint32_t IDESC_SS = instr_desc(FMT, FMT, 0u, 128, 128);
+  static constexpr uint32_t IDESC_SS64 = instr_desc(FMT, FMT, 0u, 128, 64);  // one 64-column half
   static constexpr uint32_t IDESC_TS = instr_desc(FMT, FMT, 1u, 128, D);
   static constexpr uint32_t SWZ = SW == 128 ? 2u : 4u;
   static constexpr uint32_t COL_A = 0, COL_B = 128, COL_ACC0 = 256, COL_ACC1 = 256 + D;
 };
 
-// Barrier slots: fixed tiles loaded, fixed tiles released, ring full/empty,
-// scores ready, P/dS ready, accumulators final.
+// Barrier slots: fixed tiles loaded, ring full/empty, scores of column half h
+// ready (MMA -> the four compute warps of half h), P/dS of half h ready
+// (those warps -> MMA), accumulators final, all MMAs complete.
 template <int NS>
 struct BwdBars {
   uint32_t base;
   __device__ __forceinline__ uint32_t fixed_full() const { return base; }
   __device__ __forceinline__ uint32_t full(int s) const { return base + 8u * (1 + s); }
   __device__ __forceinline__ uint32_t empty(int s) const { return base + 8u * (1 + NS + s); }
-  __device__ __forceinline__ uint32_t s_full() const { return base + 8u * (1 + 2 * NS); }
-  __device__ __forceinline__ uint32_t p_full() const { return base + 8u * (2 + 2 * NS); }
-  __device__ __forceinline__ uint32_t acc_full() const { return base + 8u * (3 + 2 * NS); }
-  __device__ __forceinline__ uint32_t mma_done() const { return base + 8u * (4 + 2 * NS); }
+  __device__ __forceinline__ uint32_t s_full(int h) const { return base + 8u * (1 + 2 * NS + h); }
+  __device__ __forceinline__ uint32_t p_full(int h) const { return base + 8u * (3 + 2 * NS + h); }
+  __device__ __forceinline__ uint32_t acc_full() const { return base + 8u * (5 + 2 * NS); }
+  __device__ __forceinline__ uint32_t mma_done() const { return base + 8u * (6 + 2 * NS); }
 };
 
 // ---------------------------------------------------------------- D pre-pass
@@ -143,6 +145,34 @@ __device__ __forceinline__ void bwd_mma_ss(uint32_t d_tmem, uint32_t a_smem, uin
   for (int kk = 0; kk < C::K_STEPS; ++kk) {
     const uint32_t off = ((kk * 32) / C::SW) * (128 * C::SW) + ((kk * 32) % C::SW);
     mma_f16_ss(d_tmem, da + (off >> 4), db + (off >> 4), C::IDESC_SS, kk > 0);
+  }
+}
+
+// The same for rows 64h..64h+63 of B only (N = 64): one column half of the
+// 128 x 128 product, written to d_tmem (the caller adds 64h).
+template <int D, int ELEM>
+__device__ __forceinline__ void bwd_mma_ss_half(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem, int h) {
+  using C = BwdCfg<D, ELEM>;
+  const uint64_t da = smem_desc(a_smem, 16, 8 * C::SW, C::SWZ);
+  const uint64_t db = smem_desc(b_smem + 64u * C::SW * h, 16, 8 * C::SW, C::SWZ);  // row 64h of each chunk
+#pragma unroll
+  for (int kk = 0; kk < C::K_STEPS; ++kk) {
+    const uint32_t off = ((kk * 32) / C::SW) * (128 * C::SW) + ((kk * 32) % C::SW);
+    mma_f16_ss(d_tmem, da + (off >> 4), db + (off >> 4), C::IDESC_SS64, kk > 0);
+  }
+}
+
+// acc (+)= A_h B_h over K rows 64h..64h+63 only (one half of bwd_mma_ts).
+template <int D, int ELEM>
+__device__ __forceinline__ void bwd_mma_ts_half(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, int h,
+                                                bool accumulate) {
+  using C = BwdCfg<D, ELEM>;
+  const uint64_t db = smem_desc(b_smem, 128 * C::SW, 8 * C::SW, C::SWZ);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int kk = 4 * h + k;
+    const uint32_t a_col = kk * 8 + (kk >= 4 ? 32u : 0u);  // packed layout as in bwd_mma_ts
+    mma_f16_ts(d_tmem, a_tmem + a_col, db + ((kk * 16 * C::SW) >> 4), C::IDESC_TS, (accumulate || k > 0) ? 1u : 0u);
   }
 }
 
@@ -228,8 +258,10 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(b.full(s), 1);
       mbar_init(b.empty(s), 1);
     }
-    mbar_init(b.s_full(), 1);
-    mbar_init(b.p_full(), 8);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(b.s_full(h), 1);
+      mbar_init(b.p_full(h), 4);  // the four compute warps of column half h
+    }
     mbar_init(b.acc_full(), 1);
     mbar_init(b.mma_done(), 1);
     fence_barrier_init();
@@ -274,25 +306,48 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else if (warp == 9) {
     if (lane == 0) {
-      bool ok = wait_bounded(b.fixed_full(), 0, abort_flag, limit);
-      for (int t = 0; t < n_i && ok; ++t) {
-        const int s = t % C::NS;
-        if (!wait_bounded(b.full(s), (t / C::NS) & 1, abort_flag, limit)) {
-          ok = false;
-          break;
-        }
+      // Per query half h (64 columns): S^T_h, dP^T_h -> the half's warps ->
+      // dV, dK += their half of the products.  While one half's warps
+      // compute, the tensor cores run the other half's accumulation and the
+      // next tile's scores for that half (issue order keeps each half's
+      // tensor-memory reuse safe).
+      auto issue_scores = [&](int s, int h) {
         const uint32_t sQ = sRing + s * C::STAGE, sDO = sQ + C::TILE;
-        bwd_mma_ss<D, ELEM>(tmem + C::COL_A, sK, sQ);   // S^T = K Q^T
-        bwd_mma_ss<D, ELEM>(tmem + C::COL_B, sV, sDO);  // dP^T = V dO^T
-        tc_commit(b.s_full());
-        if (!wait_bounded(b.p_full(), t & 1, abort_flag, limit)) {
-          ok = false;
-          break;
+        bwd_mma_ss_half<D, ELEM>(tmem + C::COL_A + 64 * h, sK, sQ, h);   // S^T_h = K Q_h^T
+        bwd_mma_ss_half<D, ELEM>(tmem + C::COL_B + 64 * h, sV, sDO, h);  // dP^T_h = V dO_h^T
+        tc_commit(b.s_full(h));
+      };
+      bool ok = wait_bounded(b.fixed_full(), 0, abort_flag, limit);
+      if (ok && n_i > 0) {
+        ok = wait_bounded(b.full(0), 0, abort_flag, limit);
+        if (ok) {
+          tc_fence_after();
+          issue_scores(0, 0);
+          issue_scores(0, 1);
         }
-        tc_fence_after();
-        bwd_mma_ts<D, ELEM>(tmem + C::COL_ACC0, tmem + C::COL_A, sDO, t > 0);  // dV += P^T dO
-        bwd_mma_ts<D, ELEM>(tmem + C::COL_ACC1, tmem + C::COL_B, sQ, t > 0);   // dK += dS^T Q
-        tc_commit(b.empty(s));
+      }
+      for (int t = 0; t < n_i && ok; ++t) {
+        const int s = t % C::NS, s1 = (t + 1) % C::NS;
+        const uint32_t sQ = sRing + s * C::STAGE, sDO = sQ + C::TILE;
+        const bool next = t + 1 < n_i;
+        for (int h = 0; h < 2 && ok; ++h) {
+          if (!wait_bounded(b.p_full(h), t & 1, abort_flag, limit)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          bwd_mma_ts_half<D, ELEM>(tmem + C::COL_ACC0, tmem + C::COL_A, sDO, h, t > 0 || h > 0);  // dV += P^T_h dO_h
+          bwd_mma_ts_half<D, ELEM>(tmem + C::COL_ACC1, tmem + C::COL_B, sQ, h, t > 0 || h > 0);   // dK += dS^T_h Q_h
+          if (h == 1) tc_commit(b.empty(s));
+          if (next) {
+            if (h == 0 && !wait_bounded(b.full(s1), ((t + 1) / C::NS) & 1, abort_flag, limit)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_scores(s1, h);
+          }
+        }
       }
       if (ok) tc_commit(b.acc_full());
       if (!ok) {
@@ -340,7 +395,7 @@ __global__ void __launch_bounds__(320, 1)
       }
       __syncwarp();
       prefetch(t + 1);  // in flight while this block computes
-      ok = __all_sync(0xffffffffu, wait_bounded(b.s_full(), t & 1, abort_flag, limit));
+      ok = __all_sync(0xffffffffu, wait_bounded(b.s_full(half), t & 1, abort_flag, limit));
       if (!ok) break;
       tc_fence_after();
 #pragma unroll 1
@@ -382,7 +437,7 @@ __global__ void __launch_bounds__(320, 1)
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(b.p_full());
+      if (lane == 0) mbar_arrive(b.p_full(half));
     }
     if (ok) ok = __all_sync(0xffffffffu, wait_bounded(b.acc_full(), 0, abort_flag, limit));
     if (ok) {
@@ -434,8 +489,10 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(b.full(s), 1);
       mbar_init(b.empty(s), 1);
     }
-    mbar_init(b.s_full(), 1);
-    mbar_init(b.p_full(), 8);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(b.s_full(h), 1);
+      mbar_init(b.p_full(h), 4);  // the four compute warps of column half h
+    }
     mbar_init(b.acc_full(), 1);
     mbar_init(b.mma_done(), 1);
     fence_barrier_init();
@@ -480,24 +537,43 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else if (warp == 9) {
     if (lane == 0) {
-      bool ok = wait_bounded(b.fixed_full(), 0, abort_flag, limit);
-      for (int t = 0; t < n_j && ok; ++t) {
-        const int s = t % C::NS;
-        if (!wait_bounded(b.full(s), (t / C::NS) & 1, abort_flag, limit)) {
-          ok = false;
-          break;
-        }
+      // Per key half h (64 columns), pipelined as in the dK/dV kernel.
+      auto issue_scores = [&](int s, int h) {
         const uint32_t sK = sRing + s * C::STAGE, sV = sK + C::TILE;
-        bwd_mma_ss<D, ELEM>(tmem + C::COL_A, sQ, sK);   // S = Q K^T
-        bwd_mma_ss<D, ELEM>(tmem + C::COL_B, sDO, sV);  // dP = dO V^T
-        tc_commit(b.s_full());
-        if (!wait_bounded(b.p_full(), t & 1, abort_flag, limit)) {
-          ok = false;
-          break;
+        bwd_mma_ss_half<D, ELEM>(tmem + C::COL_A + 64 * h, sQ, sK, h);   // S_h = Q K_h^T
+        bwd_mma_ss_half<D, ELEM>(tmem + C::COL_B + 64 * h, sDO, sV, h);  // dP_h = dO V_h^T
+        tc_commit(b.s_full(h));
+      };
+      bool ok = wait_bounded(b.fixed_full(), 0, abort_flag, limit);
+      if (ok && n_j > 0) {
+        ok = wait_bounded(b.full(0), 0, abort_flag, limit);
+        if (ok) {
+          tc_fence_after();
+          issue_scores(0, 0);
+          issue_scores(0, 1);
         }
-        tc_fence_after();
-        bwd_mma_ts<D, ELEM>(tmem + C::COL_ACC0, tmem + C::COL_A, sK, t > 0);  // dQ += dS K
-        tc_commit(b.empty(s));
+      }
+      for (int t = 0; t < n_j && ok; ++t) {
+        const int s = t % C::NS, s1 = (t + 1) % C::NS;
+        const uint32_t sK = sRing + s * C::STAGE;
+        const bool next = t + 1 < n_j;
+        for (int h = 0; h < 2 && ok; ++h) {
+          if (!wait_bounded(b.p_full(h), t & 1, abort_flag, limit)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          bwd_mma_ts_half<D, ELEM>(tmem + C::COL_ACC0, tmem + C::COL_A, sK, h, t > 0 || h > 0);  // dQ += dS_h K_h
+          if (h == 1) tc_commit(b.empty(s));
+          if (next) {
+            if (h == 0 && !wait_bounded(b.full(s1), ((t + 1) / C::NS) & 1, abort_flag, limit)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_scores(s1, h);
+          }
+        }
       }
       if (ok) tc_commit(b.acc_full());
       if (!ok) {
@@ -520,7 +596,7 @@ __global__ void __launch_bounds__(320, 1)
     const float dlt = row_ok ? a.delta[static_cast<size_t>(bh) * a.N + qrow] : 0.f;
     bool ok = true;
     for (int t = 0; t < n_j && ok; ++t) {
-      ok = __all_sync(0xffffffffu, wait_bounded(b.s_full(), t & 1, abort_flag, limit));
+      ok = __all_sync(0xffffffffu, wait_bounded(b.s_full(half), t & 1, abort_flag, limit));
       if (!ok) break;
       tc_fence_after();
       const int kb = 128 * t;
@@ -550,7 +626,7 @@ __global__ void __launch_bounds__(320, 1)
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(b.p_full());
+      if (lane == 0) mbar_arrive(b.p_full(half));
     }
     if (ok) ok = __all_sync(0xffffffffu, wait_bounded(b.acc_full(), 0, abort_flag, limit));
     if (ok) {
