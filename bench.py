@@ -313,7 +313,9 @@ def run_ours(args, rank, world, local_rank):
                                    "other cases' kernels"}
 
     # ---- per-workload suite (rank 0 only, single GPU numbers)
-    if not args.no_suite and rank == 0:
+    # single-GPU context only: with several ranks the others would sit at the
+    # final barrier for the suite's minute or more
+    if not args.no_suite and world == 1:
         suite = {}
         for name, w in WORKLOADS.items():
             if name in (args.workload, "tiny"):
