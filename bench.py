@@ -459,26 +459,32 @@ def run_ours(args, rank, world, local_rank):
         from tiled_attention_12_b200.ring import ring_attention_emulated
 
         rc = WORKLOADS["b1h32n32768d128_causal"].cases[0]
-        name = "ring8_emulated_" + rc.name
-        try:
-            q, k, v = device_inputs(rc, salt=4)
-            for _ in range(2):
-                ring_attention_emulated(q, k, v, 8, rc.causal, rc.softmax_scale)
-            times = []
-            for _ in range(3):
-                flush.zero_()
-                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a0.record(stream)
-                ring_attention_emulated(q, k, v, 8, rc.causal, rc.softmax_scale)
-                a1.record(stream)
-                torch.cuda.synchronize()
-                times.append(a0.elapsed_time(a1))
-            ms = statistics.median(times)
-            suite[name] = {"ms": round(ms, 4), "tflops": round(rc.flops / ms / 1e9, 1),
-                           "note": "ring of 8 sequence blocks run on one GPU; includes block copies and merges"}
-            del q, k, v
-        except Exception as e:  # report, never hide
-            suite[name] = {"error": str(e)[:200]}
+        for zz in (False, True):
+            name = ("ring8_zigzag_emulated_" if zz else "ring8_emulated_") + rc.name
+            try:
+                q, k, v = device_inputs(rc, salt=4)
+                for _ in range(2):
+                    ring_attention_emulated(q, k, v, 8, rc.causal, rc.softmax_scale, zigzag=zz)
+                times, ranks = [], []
+                for _ in range(3):
+                    flush.zero_()
+                    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a0.record(stream)
+                    ring_attention_emulated(q, k, v, 8, rc.causal, rc.softmax_scale, zigzag=zz)
+                    a1.record(stream)
+                    torch.cuda.synchronize()
+                    times.append(a0.elapsed_time(a1))
+                rank_ms = []
+                ring_attention_emulated(q, k, v, 8, rc.causal, rc.softmax_scale, zigzag=zz, rank_ms=rank_ms)
+                ms = statistics.median(times)
+                suite[name] = {"ms": round(ms, 4), "tflops": round(rc.flops / ms / 1e9, 1),
+                               "rank_ms_max": round(max(rank_ms), 4),
+                               "rank_ms_mean": round(sum(rank_ms) / len(rank_ms), 4),
+                               "note": "ring of 8 sequence blocks run one rank after another on one GPU; "
+                                       "includes block copies and merges; rank_ms = each rank's device time"}
+                del q, k, v
+            except Exception as e:  # report, never hide
+                suite[name] = {"error": str(e)[:200]}
         torch.cuda.synchronize()
         if fa.fa_last_device_status() != 0:
             raise SystemExit("device status reports a timed-out wait in the suite")

@@ -76,6 +76,31 @@ def test_emulated_ring_against_oracle(d, world, causal):
     gate(o, ro, lse, rl, tol=TOL_16, what=f"ring d{d} w{world} c{causal}")
 
 
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("world", [2, 4])
+def test_emulated_zigzag_ring_against_oracle(world, causal):
+    case = Case("ring_zz", 1, 4, 2048, 128, causal, seed=world + 40)
+    q, k, v = make_qkv(case)
+    o, lse = ring_attention_emulated(q.to(DEV), k.to(DEV), v.to(DEV), world, causal, zigzag=True)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status() == 0
+    ro, rl = attention_ref(q, k, v, case.softmax_scale, causal)
+    gate(o, ro, lse, rl, tol=TOL_16, what=f"zigzag ring w{world} c{causal}")
+
+
+def test_zigzag_balances_causal_work():
+    """Per-rank device time of the emulated causal ring: the zig-zag layout
+    evens it out (the contiguous one leaves the last rank with ~2x the mean)."""
+    case = Case("ring_bal", 1, 8, 16384, 128, True, seed=3)
+    q, k, v = (t.to(DEV) for t in make_qkv(case))
+    for _ in range(2):
+        cont, zz = [], []
+        ring_attention_emulated(q, k, v, 8, True, rank_ms=cont)
+        ring_attention_emulated(q, k, v, 8, True, zigzag=True, rank_ms=zz)
+    bal = lambda t: (sum(t) / len(t)) / max(t)  # noqa: E731
+    assert bal(zz) > 0.85 and bal(cont) < 0.7, (cont, zz)
+
+
 def test_emulated_ring_long_sequence():
     """B1 H8 N32768 d128 causal over 8 emulated ranks, sampled rows."""
     case = Case("ring_long", 1, 8, 32768, 128, True, seed=5)

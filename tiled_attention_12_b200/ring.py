@@ -22,6 +22,14 @@ posts the same transfers in the same order; there is no other collective.
 ``attend`` and ``merge`` default to the CUDA library (fa_fwd,
 fa_merge_partial); tests on CPU replace them to exercise the transfer
 schedule with the gloo backend.
+
+Zig-zag layout (``zigzag=True``, for the causal mask): with contiguous blocks
+rank world-1 attends to every block and rank 0 to one, so the causal work is
+unbalanced.  Cutting the sequence into 2*world chunks and giving rank r the
+chunks r and 2*world-1-r (stacked as its [B, H, 2c, d] block) equalises it.
+Each pair of (query chunk, key chunk) is again full, causal (same chunk) or
+empty (a later key chunk), so every piece is one plain fa_fwd call, merged
+into the accumulator of its query chunk.
 """
 
 from __future__ import annotations
@@ -41,6 +49,26 @@ def ring_steps(rank: int, world: int, causal: bool):
         else:
             steps.append((src, "full"))
     return steps
+
+
+def chunk_pairs(rank: int, src: int, world: int, zigzag: bool, causal: bool):
+    """Pieces of one ring step: [(query part, key part, mode)] where a part
+    indexes the rank's block (0: the whole block, or with zigzag 0/1: its
+    first/second chunk) and mode is "full" or "causal" (empty pieces are left
+    out)."""
+    if not zigzag or not causal:  # without the mask the whole block pair is one full piece
+        mode = "causal" if causal and src == rank else "full"
+        return [] if causal and src > rank else [(None, None, mode)]
+    own = (rank, 2 * world - 1 - rank)
+    other = (src, 2 * world - 1 - src)
+    pieces = []
+    for qa, qc in enumerate(own):
+        for kb, kc in enumerate(other):
+            if not causal or kc < qc:
+                pieces.append((qa, kb, "full"))
+            elif kc == qc:
+                pieces.append((qa, kb, "causal"))
+    return pieces
 
 
 def _cuda_attend(q, k, v, causal, softmax_scale):
@@ -72,24 +100,44 @@ class _Accumulator:
         self.count += 1
 
 
-def _run_steps(q, blocks, steps, causal, softmax_scale, attend, merge, out):
-    """Attend q to each block of `steps` (block fetched by blocks(i)) and merge;
-    the last contributing step writes the 16-bit result into `out`."""
-    acc = _Accumulator(q, merge)
-    live = [i for i, (_, mode) in enumerate(steps) if mode != "skip"]
-    for i, (_, mode) in enumerate(steps):
+def _run_steps(q, blocks, pieces, softmax_scale, attend, merge, out):
+    """Attend the rank's query block to the key/value block each step brings
+    (blocks(i)), piece by piece (pieces[i] from chunk_pairs), merging into one
+    accumulator per query part; each part's last piece writes its 16-bit rows
+    into `out`.  Returns (out, lse)."""
+    import torch
+
+    n_parts = 1 if all(p[0] is None for ps in pieces for p in ps) else 2
+    c = q.shape[2] // n_parts
+    # chunk views, no copies: the attention call takes strided views
+    qs = [q] if n_parts == 1 else [q[:, :, :c], q[:, :, c:]]
+    outs = [out] if n_parts == 1 else [torch.empty_like(qs[0]), torch.empty_like(qs[1])]
+    accs = [_Accumulator(x, merge) for x in qs]
+    last = {}
+    for i, ps in enumerate(pieces):
+        for p in ps:
+            last[p[0] or 0] = (i, p)
+    for i, ps in enumerate(pieces):
         k, v = blocks(i)
-        if mode == "skip":
-            continue
-        o_part, lse_part = attend(q, k, v, mode == "causal", softmax_scale)
-        acc.add(o_part, lse_part, out if i == live[-1] else None)
-    return out, acc.lse
+        for p in ps:
+            qa, kb, mode = p
+            qa = qa or 0
+            kk, vv = (k, v) if kb is None else (k[:, :, kb * c:(kb + 1) * c], v[:, :, kb * c:(kb + 1) * c])
+            o_part, lse_part = attend(qs[qa], kk, vv, mode == "causal", softmax_scale)
+            accs[qa].add(o_part, lse_part, outs[qa] if last[qa] == (i, p) else None)
+    if n_parts == 1:
+        return out, accs[0].lse
+    out[:, :, :c] = outs[0]
+    out[:, :, c:] = outs[1]
+    return out, torch.cat((accs[0].lse, accs[1].lse), dim=2)
 
 
-def ring_attention(q, k, v, causal: bool = False, softmax_scale=None, group=None, attend=None, merge=None):
+def ring_attention(q, k, v, causal: bool = False, softmax_scale=None, group=None, attend=None, merge=None,
+                   zigzag: bool = False):
     """This rank's rows of softmax(scale Q K^T [+ causal]) V over the whole
-    ring's sequence.  q, k, v: this rank's [B, H, n, d] contiguous blocks.
-    Returns (o [B, H, n, d] in q's dtype, lse [B, H, n] fp32)."""
+    ring's sequence.  q, k, v: this rank's [B, H, n, d] contiguous blocks
+    (zigzag: its two chunks stacked, n even).  Returns (o [B, H, n, d] in q's
+    dtype, lse [B, H, n] fp32) for the same rows."""
     import torch
     import torch.distributed as dist
 
@@ -98,6 +146,7 @@ def ring_attention(q, k, v, causal: bool = False, softmax_scale=None, group=None
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
     steps = ring_steps(rank, world, causal)
+    pieces = [chunk_pairs(rank, src, world, zigzag, causal) for src, _ in steps]
     nxt = dist.get_global_rank(group, (rank + 1) % world) if group is not None else (rank + 1) % world
     prv = dist.get_global_rank(group, (rank - 1) % world) if group is not None else (rank - 1) % world
 
@@ -117,36 +166,51 @@ def ring_attention(q, k, v, causal: bool = False, softmax_scale=None, group=None
         return cur[0], cur[1]
 
     out = torch.empty_like(q)
-    o, lse = _run_steps(q, blocks, steps, causal, softmax_scale, attend, merge, out)
+    o, lse = _run_steps(q, blocks, pieces, softmax_scale, attend, merge, out)
     if pending[0] is not None:
         for req in pending[0]:
             req.wait()
     return o, lse
 
 
-def ring_attention_emulated(q, k, v, world: int, causal: bool = False, softmax_scale=None):
-    """The ring on one device: the full [B, H, N, d] tensors are cut into
-    `world` equal sequence blocks and every rank's steps run one after the
-    other (no rank waits on another).  Returns (o, lse) for the whole
-    sequence.  It runs exactly the per-rank attention and merge calls of
-    ring_attention, without the transfers."""
+def ring_attention_emulated(q, k, v, world: int, causal: bool = False, softmax_scale=None, zigzag: bool = False,
+                            rank_ms=None):
+    """The ring on one device: the full [B, H, N, d] tensors are cut into the
+    ranks' blocks (contiguous, or zig-zag chunk pairs) and every rank's steps
+    run one after the other (no rank waits on another).  It runs exactly the
+    per-rank attention and merge calls of ring_attention, without the
+    transfers.  With ``rank_ms`` a list, each rank's device time (CUDA events)
+    is appended to it: the maximum is the compute time of a real ring.
+    Returns (o, lse) for the whole sequence."""
     import torch
 
     B, H, N, d = q.shape
-    if N % world:
+    parts = 2 * world if zigzag else world
+    if N % parts:
         raise ValueError("the sequence length must split into equal blocks")
-    n = N // world
-    blk = [slice(r * n, (r + 1) * n) for r in range(world)]
+    c = N // parts
+    if zigzag:
+        rows = [torch.cat((torch.arange(r * c, (r + 1) * c), torch.arange((parts - 1 - r) * c, (parts - r) * c)))
+                for r in range(world)]
+    else:
+        rows = [torch.arange(r * c, (r + 1) * c) for r in range(world)]
+    rows = [r.to(q.device) for r in rows]
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
+    blk = {r: (k[:, :, rows[r]].contiguous(), v[:, :, rows[r]].contiguous()) for r in range(world)}
     for rank in range(world):
         steps = ring_steps(rank, world, causal)
-        qr = q[:, :, blk[rank]].contiguous()
-        kv = {src: (k[:, :, blk[src]].contiguous(), v[:, :, blk[src]].contiguous())
-              for src, mode in steps if mode != "skip"}
+        pieces = [chunk_pairs(rank, src, world, zigzag, causal) for src, _ in steps]
+        qr = q[:, :, rows[rank]].contiguous()
         out = torch.empty_like(qr)
-        _, lr = _run_steps(qr, lambda i: kv.get(steps[i][0], (None, None)), steps, causal, softmax_scale,
-                           _cuda_attend, _cuda_merge, out)
-        o[:, :, blk[rank]] = out
-        lse[:, :, blk[rank]] = lr
+        if rank_ms is not None:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+        _, lr = _run_steps(qr, lambda i: blk[steps[i][0]], pieces, softmax_scale, _cuda_attend, _cuda_merge, out)
+        if rank_ms is not None:
+            e1.record()
+            torch.cuda.synchronize()
+            rank_ms.append(e0.elapsed_time(e1))
+        o[:, :, rows[rank]] = out
+        lse[:, :, rows[rank]] = lr
     return o, lse
