@@ -88,6 +88,12 @@ WORKLOADS = {
         _c("b4h16n8192d128", 4, 16, 8192, 128, False, 2, value_scale=0.5),
         _c("b1h32n16384d128", 1, 32, 16384, 128, False, 5),),
         "B=4 H=16 N=8192 d=128 and B=1 H=32 N=16384 d=128, non-causal"),
+    # the middle head size (the pages' tiny config uses d = 64): same shape as
+    # the d_model 512 comparison, twice the head width (d_model 1024)
+    "b1h16n16384d64": Workload("b1h16n16384d64", (
+        _c("b1h16n16384d64_causal", 1, 16, 16384, 64, True, 6),
+        _c("b1h16n16384d64", 1, 16, 16384, 64, False, 6),),
+        "B=1 H=16 N=16384 d=64, causal and non-causal, N(0,1)"),
 }
 
 
