@@ -168,11 +168,19 @@ def run_ours(args, rank, world, local_rank):
     # inputs resident in HBM (same recipe as synth.make_qkv, drawn on the
     # device with a rank-specific seed: each rank holds its own batch)
     def device_inputs(case, salt=0):
+        """The case's recipe drawn on the device: N(0,1) times the multiplier,
+        and the outlier mask (each entry independently) where the case has one."""
         g = torch.Generator(device=dev)
         g.manual_seed(case.seed * 1009 + rank * 7919 + salt)
         shape = (case.B, case.H, case.N, case.d)
-        return [(torch.randn(shape, generator=g, device=dev) * case.value_scale).to(torch.bfloat16)
-                for _ in range(3)]
+        out = []
+        for _ in range(3):
+            t = torch.randn(shape, generator=g, device=dev)
+            if case.outlier_frac > 0:
+                t = torch.where(torch.rand(shape, generator=g, device=dev) < case.outlier_frac,
+                                t * case.outlier_mult, t)
+            out.append((t * case.value_scale).to(torch.bfloat16))
+        return out
 
     cases = [c for c in wl.cases if args.only_case in (None, c.name)]
     if not cases:
