@@ -21,9 +21,12 @@
 //                      once more) avoids fp32 atomics on dQ.
 //
 // Warps 0-7: compute (warp w: rows 32(w%4)..+31 of the 128-row tile, columns
-// 64(w/4)..+63 of the 128x128 score block; two warps per scheduler partition
-// keep the exp2 unit busy); warp 8: TMA producer; warp 9: tensor-memory
-// allocation and the MMA-issuing thread.
+// 64(w/4)..+63 of the 128x128 score block); warp 8: TMA producer; warp 9:
+// tensor-memory allocation and the MMA-issuing thread.  Both kernels are
+// pipelined by column half: the scores of each 64-column half are issued as
+// their own N = 64 products with their own barrier, the half's four warps
+// hand P/dS back on another, and the MMA thread accumulates that half and
+// issues the next block's scores for it while the other half computes.
 // Tensor memory (dK/dV kernel): S^T [0,128), dP^T [128,256), dV [256,256+d),
 // dK [256+d,256+2d); (dQ kernel): S [0,128), dP [128,256), dQ [256,256+d).
 // Every wait is bounded as in the forward kernel.
@@ -76,8 +79,7 @@ struct BwdCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget exceeded");
   static constexpr int K_STEPS = ROW / 32;                    // 16 elements per MMA K step
   static constexpr uint32_t FMT = ELEM == 1 ? 0u : 1u;        // f16 : bf16
-  static constexpr uint32_t IDESC_SS = instr_desc(FMT, FMT, 0u, 128, 128);
-  static constexpr uint32_t IDESC_SS64 = instr_desc(FMT, FMT, 0u, 128, 64);  // one 64-column half
+  static constexpr uint32_t IDESC_SS64 = instr_desc(FMT, FMT, 0u, 128, 64);  // one 64-column half of S / dP
   static constexpr uint32_t IDESC_TS = instr_desc(FMT, FMT, 1u, 128, D);
   static constexpr uint32_t SWZ = SW == 128 ? 2u : 4u;
   static constexpr uint32_t COL_A = 0, COL_B = 128, COL_ACC0 = 256, COL_ACC1 = 256 + D;
@@ -135,21 +137,9 @@ __device__ __forceinline__ void bwd_load_tile(uint32_t dst, const CUtensorMap* m
     tma_load_3d(dst + c * 128 * C::SW, map, bar, c * (C::SW / 2), row0, bh);
 }
 
-// A x B^T with both operands K-major 128-row tiles in shared memory.
-template <int D, int ELEM>
-__device__ __forceinline__ void bwd_mma_ss(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
-  using C = BwdCfg<D, ELEM>;
-  const uint64_t da = smem_desc(a_smem, 16, 8 * C::SW, C::SWZ);
-  const uint64_t db = smem_desc(b_smem, 16, 8 * C::SW, C::SWZ);
-#pragma unroll
-  for (int kk = 0; kk < C::K_STEPS; ++kk) {
-    const uint32_t off = ((kk * 32) / C::SW) * (128 * C::SW) + ((kk * 32) % C::SW);
-    mma_f16_ss(d_tmem, da + (off >> 4), db + (off >> 4), C::IDESC_SS, kk > 0);
-  }
-}
-
-// The same for rows 64h..64h+63 of B only (N = 64): one column half of the
-// 128 x 128 product, written to d_tmem (the caller adds 64h).
+// A x B^T over rows 64h..64h+63 of B (N = 64): one column half of the
+// 128 x 128 product of two K-major 128-row tiles in shared memory, written
+// to d_tmem (the caller adds 64h).
 template <int D, int ELEM>
 __device__ __forceinline__ void bwd_mma_ss_half(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem, int h) {
   using C = BwdCfg<D, ELEM>;
@@ -162,7 +152,11 @@ __device__ __forceinline__ void bwd_mma_ss_half(uint32_t d_tmem, uint32_t a_smem
   }
 }
 
-// acc (+)= A_h B_h over K rows 64h..64h+63 only (one half of bwd_mma_ts).
+// acc (+)= A_h B_h: A (128 x 128, 16-bit, packed) in tensor memory at
+// a_tmem, B a 128-row tile in shared memory read N-major (its rows are the K
+// index); only K rows 64h..64h+63.  The packed A keeps K rows 0..63 at
+// columns 0..31 and rows 64..127 at columns 64..95 (each compute warp packs
+// inside its own 64-column half).
 template <int D, int ELEM>
 __device__ __forceinline__ void bwd_mma_ts_half(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, int h,
                                                 bool accumulate) {
@@ -171,23 +165,8 @@ __device__ __forceinline__ void bwd_mma_ts_half(uint32_t d_tmem, uint32_t a_tmem
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int kk = 4 * h + k;
-    const uint32_t a_col = kk * 8 + (kk >= 4 ? 32u : 0u);  // packed layout as in bwd_mma_ts
-    mma_f16_ts(d_tmem, a_tmem + a_col, db + ((kk * 16 * C::SW) >> 4), C::IDESC_TS, (accumulate || k > 0) ? 1u : 0u);
-  }
-}
-
-// acc (+)= A B with A (128 x 128, 16-bit) in tensor memory at a_tmem and B a
-// 128-row tile in shared memory read N-major (its rows are the K index).
-template <int D, int ELEM>
-__device__ __forceinline__ void bwd_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, bool accumulate) {
-  using C = BwdCfg<D, ELEM>;
-  const uint64_t db = smem_desc(b_smem, 128 * C::SW, 8 * C::SW, C::SWZ);
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    // packed 16-bit operand: rows 0..63 of K at columns 0..31, rows 64..127 at
-    // columns 64..95 (each compute warp packs inside its own 64-column half)
     const uint32_t a_col = kk * 8 + (kk >= 4 ? 32u : 0u);
-    mma_f16_ts(d_tmem, a_tmem + a_col, db + ((kk * 16 * C::SW) >> 4), C::IDESC_TS, (accumulate || kk > 0) ? 1u : 0u);
+    mma_f16_ts(d_tmem, a_tmem + a_col, db + ((kk * 16 * C::SW) >> 4), C::IDESC_TS, (accumulate || k > 0) ? 1u : 0u);
   }
 }
 
