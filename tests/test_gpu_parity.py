@@ -157,7 +157,7 @@ def _full_or_sampled(case: Case, dtype=torch.bfloat16, max_full_flops=2e10):
 
 
 @pytest.mark.parametrize("case", [c for w in ("tiny", "dmodel512_h16", "b4h16n8192d128_causal",
-                                              "b1h32n32768d128_causal", "target_d128_noncausal")
+                                              "b1h32n32768d128_causal", "target_d128_noncausal", "b1h16n16384d64")
                                   for c in WORKLOADS[w].cases], ids=lambda c: c.name)
 def test_named_workload(case):
     _full_or_sampled(case)
