@@ -50,6 +50,8 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true", help="skip the oracle baseline")
     p.add_argument("--only-case", default=None, help="time one case of the workload (profiling)")
+    p.add_argument("--clock-log", default=None,
+                   help="path prefix for the nvidia-smi clock samples (default: a temporary file)")
     return p.parse_args()
 
 
@@ -221,8 +223,7 @@ def run_ours(args, rank, world, local_rank):
     n_cases = len(cases)
     ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(n_cases)] for _ in range(args.steps)]
-    sampler = ClockSampler(local_rank, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
-                           if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else None)
+    sampler = ClockSampler(local_rank, f"{args.clock_log}.rank{rank}.csv" if args.clock_log else None)
     time.sleep(0.3)
     barrier()
     torch.cuda.synchronize()
