@@ -581,13 +581,8 @@ __global__ void __launch_bounds__(320, 1)
       const int kb = 128 * t;
       // keys past the sequence end, or after the query when causal, are masked
       const int limit_key = (a.causal && qrow < a.N - 1) ? qrow : a.N - 1;
-#pragma unroll 1
-      for (int c = 2 * half; c < 2 * half + 2; ++c) {
-        ChunkIn in;
-        tmem_ld32(tS + 32 * c, in.s);
-        tmem_ld32(tP + 32 * c, in.dp);
-        tmem_ld_wait(in.s);
-        reg_tie(in.dp);
+      // dS of one 32-key chunk from its S and dP columns, packed in place
+      auto chunk_ds = [&](const ChunkIn& in, int c) {
         uint32_t pd[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
@@ -601,7 +596,20 @@ __global__ void __launch_bounds__(320, 1)
           pd[e >> 1] = pack16<ELEM>(dv[0], dv[1]);
         }
         tmem_st16(tS + 64 * half + 16 * (c - 2 * half), pd);
-      }
+      };
+      // both chunks' loads in flight together: one tensor-memory latency
+      ChunkIn in0, in1;
+      tmem_ld32(tS + 64 * half, in0.s);
+      tmem_ld32(tP + 64 * half, in0.dp);
+      tmem_ld32(tS + 64 * half + 32, in1.s);
+      tmem_ld32(tP + 64 * half + 32, in1.dp);
+      tmem_ld_wait(in0.s);
+      reg_tie(in0.dp);
+      reg_tie(in1.s);
+      reg_tie(in1.dp);
+      chunk_ds(in0, 2 * half);
+      chunk_ds(in1, 2 * half + 1);
+
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
