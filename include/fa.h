@@ -142,6 +142,7 @@ fa_status fa_fwd_strided(const void* q, const void* k, const void* v, void* o, f
  *   Other arguments, layouts and dtypes as in fa_fwd.
  * A query row with no computed key gets a zero output row and LSE = -inf.
  * Ceiling: ceil(N/128) <= 512 (N <= 65536); larger N -> FA_ERR_UNSUPPORTED.
+ * dtype FA_E4M3_ALL is not offered here (FA_ERR_UNSUPPORTED).
  * The library builds a per-call plan (the K/V tiles each 256-row work tile
  * visits) in a workspace grown on demand with cudaMalloc and freed by
  * fa_release; the mask is read on `stream` before the attention kernel and
