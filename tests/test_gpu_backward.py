@@ -66,6 +66,29 @@ def test_backward_many_heads_and_blocks():
     _run(Case("bwdbig", 2, 8, 1024, 128, True, seed=6, value_scale=0.5))
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_bench_size_sampled_rows(causal):
+    """B4 H16 N8192 d128 (the shape the bench times) on sampled query and key
+    rows of two heads, against the oracle's row-sampled gradients."""
+    from oracle.backward import attention_bwd_rows
+    from parity_util import sample_rows
+    case = Case("bwd_full", 4, 16, 8192, 128, causal, seed=31, value_scale=0.5)
+    q, k, v = make_qkv(case)
+    g = make_tensor((case.B, case.H, case.N, case.d), 131)
+    qd, kd, vd, gd = q.cuda(), k.cuda(), v.cuda(), g.cuda()
+    o, lse = fa.fa_fwd(qd, kd, vd, causal=causal)
+    dq, dk, dv = fa.fa_bwd(qd, kd, vd, o, lse, gd, causal=causal)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status() == 0
+    rows = sample_rows(case.N, seed=3, n_random=32)
+    idx = torch.as_tensor(rows, device="cuda")
+    for b, h in ((0, 0), (3, 15)):
+        rq, rk, rv = attention_bwd_rows(q, k, v, g, case.softmax_scale, causal, b, h, rows, rows)
+        _check(f"dq ({b},{h})", dq[b, h][idx], rq)
+        _check(f"dk ({b},{h})", dk[b, h][idx], rk)
+        _check(f"dv ({b},{h})", dv[b, h][idx], rv)
+
+
 def test_backward_rejects_fp8_and_aliasing():
     c = Case("x", 1, 1, 128, 128, False, seed=1)
     q, k, v = (t.cuda() for t in make_qkv(c))

@@ -80,3 +80,18 @@ def test_d_prepass_equals_rowsum_of_p_dp():
     p /= p.sum(axis=1, keepdims=True)
     dp = g[0, 0] @ v[0, 0].T
     assert np.max(np.abs(dd[0, 0] - np.sum(p * dp, axis=1))) < 1e-12
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_sampled_rows_match_full_backward(causal):
+    """The row-sampled gradients equal the full ones at the sampled rows."""
+    from oracle.backward import attention_bwd_rows
+    n, d = 37, 6
+    q, k, v, g = (_rand((2, 3, n, d), s) for s in (21, 22, 23, 24))
+    dq, dk, dv = attention_bwd_ref(q, k, v, g, 0.4, causal)
+    rows = [0, 5, 17, 36]
+    for b, h in ((0, 0), (1, 2)):
+        rq, rk, rv = attention_bwd_rows(q, k, v, g, 0.4, causal, b, h, rows, rows[::-1])
+        assert np.max(np.abs(rq - dq[b, h, rows])) < 1e-12
+        assert np.max(np.abs(rk - dk[b, h, rows[::-1]])) < 1e-12
+        assert np.max(np.abs(rv - dv[b, h, rows[::-1]])) < 1e-12
