@@ -47,3 +47,16 @@ cudaError_t launch_bwd(int d, int elem, const BwdLaunch& l) {
 }
 
 }  // namespace fa
+
+#ifdef FA_TRACE
+// Trace-enabled builds only: copies the backward kernels' trace array out
+// and clears it (same record format as the forward's reader).
+extern "C" int fa_bwd_trace_read(unsigned long long* host, int cap) {
+  if (cap < FA_TRACE_CAP) return -1;
+  if (cudaMemcpyFromSymbol(host, fa::g_fa_trace, FA_TRACE_CAP * sizeof(unsigned long long)) != cudaSuccess)
+    return -1;
+  static unsigned long long zeros[FA_TRACE_CAP];
+  if (cudaMemcpyToSymbol(fa::g_fa_trace, zeros, sizeof(zeros)) != cudaSuccess) return -1;
+  return FA_TRACE_CAP;
+}
+#endif

@@ -175,6 +175,9 @@ __device__ __forceinline__ uint32_t pack16(float lo, float hi) {
   return ELEM == 1 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
 }
 
+// Mask of the n lowest bits (n in [0, 32]).
+__device__ __forceinline__ uint32_t low_bits(int n) { return n >= 32 ? 0xffffffffu : (1u << n) - 1u; }
+
 // Scores of one 32-column chunk turned into 16-bit P and dS (both written
 // back over the first half of their own regions).  Column e of the chunk is
 // the other side's row (query for dK/dV, key for dQ); `valid(e)` masks it.
@@ -261,12 +264,14 @@ __global__ void __launch_bounds__(320, 1)
       bwd_load_tile<D, ELEM>(sV, &map_v, b.fixed_full(), 128 * j, bh);
       bool ok = true;
       int issued = 0;
+      FA_TRACE_DECL;
       for (int t = 0; t < n_i && ok; ++t) {
         const int s = t % C::NS, r = t / C::NS;
         if (r > 0 && !wait_bounded(b.empty(s), (r - 1) & 1, abort_flag, limit)) {
           ok = false;
           break;
         }
+        FA_TRACE_EV(3, 90, t);
         const uint32_t dst = sRing + s * C::STAGE;
         mbar_arrive_expect_tx(b.full(s), 2 * C::TILE);
         bwd_load_tile<D, ELEM>(dst, &map_q, b.full(s), 128 * (i0 + t), bh);
@@ -296,6 +301,7 @@ __global__ void __launch_bounds__(320, 1)
         bwd_mma_ss_half<D, ELEM>(tmem + C::COL_B + 64 * h, sV, sDO, h);  // dP^T_h = V dO_h^T
         tc_commit(b.s_full(h));
       };
+      FA_TRACE_DECL;
       bool ok = wait_bounded(b.fixed_full(), 0, abort_flag, limit);
       if (ok && n_i > 0) {
         ok = wait_bounded(b.full(0), 0, abort_flag, limit);
@@ -314,10 +320,12 @@ __global__ void __launch_bounds__(320, 1)
             ok = false;
             break;
           }
+          FA_TRACE_EV(2, 60 + h, t);
           tc_fence_after();
           bwd_mma_ts_half<D, ELEM>(tmem + C::COL_ACC0, tmem + C::COL_A, sDO, h, t > 0 || h > 0);  // dV += P^T_h dO_h
           bwd_mma_ts_half<D, ELEM>(tmem + C::COL_ACC1, tmem + C::COL_B, sQ, h, t > 0 || h > 0);   // dK += dS^T_h Q_h
           if (h == 1) tc_commit(b.empty(s));
+          FA_TRACE_EV(2, 62 + h, t);
           if (next) {
             if (h == 0 && !wait_bounded(b.full(s1), ((t + 1) / C::NS) & 1, abort_flag, limit)) {
               ok = false;
@@ -325,6 +333,7 @@ __global__ void __launch_bounds__(320, 1)
             }
             tc_fence_after();
             issue_scores(s1, h);
+            FA_TRACE_EV(2, 64 + h, t + 1);
           }
         }
       }
@@ -364,6 +373,8 @@ __global__ void __launch_bounds__(320, 1)
     float* stage_l = lse_d_stage[warp][0];
     float* stage_d = lse_d_stage[warp][1];
     bool ok = true;
+    FA_TRACE_DECL;
+    const bool tr = lane == 0 && quarter == 0;
     for (int t = 0; t < n_i && ok; ++t) {
       const int qb = (i0 + t) * 128;
       __syncwarp();  // every lane is done reading the previous block's values
@@ -374,9 +385,11 @@ __global__ void __launch_bounds__(320, 1)
       }
       __syncwarp();
       prefetch(t + 1);  // in flight while this block computes
+      if (tr) FA_TRACE_EV(half, 70 + 10 * half, t);
       ok = __all_sync(0xffffffffu, wait_bounded(b.s_full(half), t & 1, abort_flag, limit));
       if (!ok) break;
       tc_fence_after();
+      if (tr) FA_TRACE_EV(half, 71 + 10 * half, t);
 #pragma unroll 1
       for (int c = 2 * half; c < 2 * half + 2; ++c) {
         ChunkIn in;
@@ -395,28 +408,45 @@ __global__ void __launch_bounds__(320, 1)
         }
         tmem_ld_wait(in.s);
         reg_tie(in.dp);
+        if (tr) FA_TRACE_EV(half, 72 + 10 * half + 2 * (c - 2 * half), t);
+        // Column e holds query q0 + e; it counts when that query exists and,
+        // if causal, does not precede this key: lo <= e < hi.  Chunks with
+        // every column valid (all but the tail and the diagonal) take the
+        // loop without selects.
+        const int hi = min(max(a.N - q0, 0), 32);
+        const int lo = a.causal ? min(max(key - q0, 0), 32) : 0;
+        const uint32_t vmask = low_bits(hi) & ~low_bits(lo);
         uint32_t pp[16], pd[16];
+        auto chunk = [&](auto masked) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float pv[2], dv[2];
+          for (int e = 0; e < 32; e += 2) {
+            float pv[2], dv[2];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int qq = q0 + e + u;
-            const bool valid = qq < a.N && !(a.causal && qq < key);
-            const float p = ex2_approx(fmaf(__uint_as_float(in.s[e + u]), a.scale_log2, -lse2[e + u]));
-            pv[u] = valid ? p : 0.f;
-            dv[u] = pv[u] * (__uint_as_float(in.dp[e + u]) - dlt[e + u]);
+            for (int u = 0; u < 2; ++u) {
+              const float p = ex2_approx(fmaf(__uint_as_float(in.s[e + u]), a.scale_log2, -lse2[e + u]));
+              if constexpr (decltype(masked)::value)
+                pv[u] = (vmask >> (e + u)) & 1u ? p : 0.f;
+              else
+                pv[u] = p;
+              dv[u] = pv[u] * (__uint_as_float(in.dp[e + u]) - dlt[e + u]);
+            }
+            pp[e >> 1] = pack16<ELEM>(pv[0], pv[1]);
+            pd[e >> 1] = pack16<ELEM>(dv[0], dv[1]);
           }
-          pp[e >> 1] = pack16<ELEM>(pv[0], pv[1]);
-          pd[e >> 1] = pack16<ELEM>(dv[0], dv[1]);
-        }
+        };
+        if (vmask == 0xffffffffu)
+          chunk(std::false_type{});
+        else
+          chunk(std::true_type{});
         tmem_st16(tS + 64 * half + 16 * (c - 2 * half), pp);
         tmem_st16(tP + 64 * half + 16 * (c - 2 * half), pd);
+        if (tr) FA_TRACE_EV(half, 73 + 10 * half + 2 * (c - 2 * half), t);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(b.p_full(half));
+      if (tr) FA_TRACE_EV(half, 76 + 10 * half, t);
     }
     if (ok) ok = __all_sync(0xffffffffu, wait_bounded(b.acc_full(), 0, abort_flag, limit));
     if (ok) {
@@ -582,19 +612,31 @@ __global__ void __launch_bounds__(320, 1)
       // keys past the sequence end, or after the query when causal, are masked
       const int limit_key = (a.causal && qrow < a.N - 1) ? qrow : a.N - 1;
       // dS of one 32-key chunk from its S and dP columns, packed in place
+      // (column e holds key kb + 32c + e: valid for e < hi; chunks with
+      // every column valid take the loop without selects)
       auto chunk_ds = [&](const ChunkIn& in, int c) {
+        const int hi = row_ok ? min(max(limit_key - kb - 32 * c + 1, 0), 32) : 0;
+        const uint32_t vmask = low_bits(hi);
         uint32_t pd[16];
+        auto body = [&](auto masked) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float dv[2];
+          for (int e = 0; e < 32; e += 2) {
+            float dv[2];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const bool valid = row_ok && kb + 32 * c + e + u <= limit_key;
-            const float p = ex2_approx(fmaf(__uint_as_float(in.s[e + u]), a.scale_log2, -lse2));
-            dv[u] = valid ? p * (__uint_as_float(in.dp[e + u]) - dlt) : 0.f;
+            for (int u = 0; u < 2; ++u) {
+              const float p = ex2_approx(fmaf(__uint_as_float(in.s[e + u]), a.scale_log2, -lse2));
+              if constexpr (decltype(masked)::value)
+                dv[u] = (vmask >> (e + u)) & 1u ? p * (__uint_as_float(in.dp[e + u]) - dlt) : 0.f;
+              else
+                dv[u] = p * (__uint_as_float(in.dp[e + u]) - dlt);
+            }
+            pd[e >> 1] = pack16<ELEM>(dv[0], dv[1]);
           }
-          pd[e >> 1] = pack16<ELEM>(dv[0], dv[1]);
-        }
+        };
+        if (hi == 32)
+          body(std::false_type{});
+        else
+          body(std::true_type{});
         tmem_st16(tS + 64 * half + 16 * (c - 2 * half), pd);
       };
       // both chunks' loads in flight together: one tensor-memory latency
