@@ -175,6 +175,13 @@ __device__ __forceinline__ uint32_t pack16(float lo, float hi) {
   return ELEM == 1 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
 }
 
+// Lane-wise product of two packed fp32 pairs (round to nearest, as mul.f32).
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 // Mask of the n lowest bits (n in [0, 32]).
 __device__ __forceinline__ uint32_t low_bits(int n) { return n >= 32 ? 0xffffffffu : (1u << n) - 1u; }
 
@@ -365,8 +372,8 @@ __global__ void __launch_bounds__(320, 1)
       for (int u = 0; u < 2; ++u) {
         const int qq = (i0 + tt) * 128 + 64 * half + 32 * u + lane;
         const bool in_seq = tt < n_i && qq < a.N;
-        pre_l[u] = in_seq ? lse_h[qq] * 1.4426950408889634f : 0.f;
-        pre_d[u] = in_seq ? dlt_h[qq] : 0.f;
+        pre_l[u] = in_seq ? -(lse_h[qq] * 1.4426950408889634f) : 0.f;  // -LSE, log2 units
+        pre_d[u] = in_seq ? -dlt_h[qq] : 0.f;                           // -D
       }
     };
     prefetch(0);
@@ -395,16 +402,16 @@ __global__ void __launch_bounds__(320, 1)
         ChunkIn in;
         tmem_ld32(tS + 32 * c, in.s);
         tmem_ld32(tP + 32 * c, in.dp);
-        // LSE (log2 units) and D of the chunk's 32 queries (the same for every lane)
+        // -LSE (log2 units) and -D of the chunk's 32 queries (the same for every lane)
         const int q0 = qb + 32 * c;
-        float lse2[32], dlt[32];
+        float nlse2[32], ndlt[32];
         const float4* sl4 = reinterpret_cast<const float4*>(stage_l + 32 * (c - 2 * half));
         const float4* sd4 = reinterpret_cast<const float4*>(stage_d + 32 * (c - 2 * half));
 #pragma unroll
         for (int v4 = 0; v4 < 8; ++v4) {
           const float4 l4 = sl4[v4], d4 = sd4[v4];
-          lse2[4 * v4] = l4.x; lse2[4 * v4 + 1] = l4.y; lse2[4 * v4 + 2] = l4.z; lse2[4 * v4 + 3] = l4.w;
-          dlt[4 * v4] = d4.x; dlt[4 * v4 + 1] = d4.y; dlt[4 * v4 + 2] = d4.z; dlt[4 * v4 + 3] = d4.w;
+          nlse2[4 * v4] = l4.x; nlse2[4 * v4 + 1] = l4.y; nlse2[4 * v4 + 2] = l4.z; nlse2[4 * v4 + 3] = l4.w;
+          ndlt[4 * v4] = d4.x; ndlt[4 * v4 + 1] = d4.y; ndlt[4 * v4 + 2] = d4.z; ndlt[4 * v4 + 3] = d4.w;
         }
         tmem_ld_wait(in.s);
         reg_tie(in.dp);
@@ -417,21 +424,26 @@ __global__ void __launch_bounds__(320, 1)
         const int lo = a.causal ? min(max(key - q0, 0), 32) : 0;
         const uint32_t vmask = low_bits(hi) & ~low_bits(lo);
         uint32_t pp[16], pd[16];
+        const uint64_t sl2x2 = pack2(a.scale_log2, a.scale_log2);
+        // two columns per packed instruction: p = 2^(s sl2 - LSE), ds = p (dp - D)
         auto chunk = [&](auto masked) {
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            float pv[2], dv[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const float p = ex2_approx(fmaf(__uint_as_float(in.s[e + u]), a.scale_log2, -lse2[e + u]));
-              if constexpr (decltype(masked)::value)
-                pv[u] = (vmask >> (e + u)) & 1u ? p : 0.f;
-              else
-                pv[u] = p;
-              dv[u] = pv[u] * (__uint_as_float(in.dp[e + u]) - dlt[e + u]);
+            const uint64_t x2 = ffma2(pack2(__uint_as_float(in.s[e]), __uint_as_float(in.s[e + 1])), sl2x2,
+                                      pack2(nlse2[e], nlse2[e + 1]));
+            float x0, x1;
+            unpack2(x2, x0, x1);
+            float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            if constexpr (decltype(masked)::value) {
+              p0 = (vmask >> e) & 1u ? p0 : 0.f;
+              p1 = (vmask >> (e + 1)) & 1u ? p1 : 0.f;
             }
-            pp[e >> 1] = pack16<ELEM>(pv[0], pv[1]);
-            pd[e >> 1] = pack16<ELEM>(dv[0], dv[1]);
+            const uint64_t d2 = fadd2(pack2(__uint_as_float(in.dp[e]), __uint_as_float(in.dp[e + 1])),
+                                      pack2(ndlt[e], ndlt[e + 1]));
+            float ds0, ds1;
+            unpack2(fmul2(pack2(p0, p1), d2), ds0, ds1);
+            pp[e >> 1] = pack16<ELEM>(p0, p1);
+            pd[e >> 1] = pack16<ELEM>(ds0, ds1);
           }
         };
         if (vmask == 0xffffffffu)
@@ -603,6 +615,8 @@ __global__ void __launch_bounds__(320, 1)
     const bool row_ok = qrow < a.N;
     const float lse2 = row_ok ? a.lse[static_cast<size_t>(bh) * a.N + qrow] * 1.4426950408889634f : 0.f;
     const float dlt = row_ok ? a.delta[static_cast<size_t>(bh) * a.N + qrow] : 0.f;
+    const uint64_t sl2x2 = pack2(a.scale_log2, a.scale_log2);
+    const uint64_t nlse2x2 = pack2(-lse2, -lse2), ndltx2 = pack2(-dlt, -dlt);
     bool ok = true;
     for (int t = 0; t < n_j && ok; ++t) {
       ok = __all_sync(0xffffffffu, wait_bounded(b.s_full(half), t & 1, abort_flag, limit));
@@ -621,16 +635,17 @@ __global__ void __launch_bounds__(320, 1)
         auto body = [&](auto masked) {
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            float dv[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const float p = ex2_approx(fmaf(__uint_as_float(in.s[e + u]), a.scale_log2, -lse2));
-              if constexpr (decltype(masked)::value)
-                dv[u] = (vmask >> (e + u)) & 1u ? p * (__uint_as_float(in.dp[e + u]) - dlt) : 0.f;
-              else
-                dv[u] = p * (__uint_as_float(in.dp[e + u]) - dlt);
+            const uint64_t x2 = ffma2(pack2(__uint_as_float(in.s[e]), __uint_as_float(in.s[e + 1])), sl2x2, nlse2x2);
+            float x0, x1;
+            unpack2(x2, x0, x1);
+            const uint64_t d2 = fadd2(pack2(__uint_as_float(in.dp[e]), __uint_as_float(in.dp[e + 1])), ndltx2);
+            float ds0, ds1;
+            unpack2(fmul2(pack2(ex2_approx(x0), ex2_approx(x1)), d2), ds0, ds1);
+            if constexpr (decltype(masked)::value) {
+              ds0 = (vmask >> e) & 1u ? ds0 : 0.f;
+              ds1 = (vmask >> (e + 1)) & 1u ? ds1 : 0.f;
             }
-            pd[e >> 1] = pack16<ELEM>(dv[0], dv[1]);
+            pd[e >> 1] = pack16<ELEM>(ds0, ds1);
           }
         };
         if (hi == 32)
