@@ -154,10 +154,12 @@ __device__ __forceinline__ void bwd_mma_ss_half(uint32_t d_tmem, uint32_t a_smem
 
 // acc (+)= A_h B_h: A (128 x 128, 16-bit, packed) in tensor memory at
 // a_tmem, B a 128-row tile in shared memory read N-major (its rows are the K
-// index); only K rows 64h..64h+63.  The packed A keeps K rows 0..63 at
-// columns 0..31 and rows 64..127 at columns 64..95 (each compute warp packs
-// inside its own 64-column half).
-template <int D, int ELEM>
+// index); only K rows 64h..64h+63.  Packed A layouts: by half (CHUNKS
+// false), K rows 0..63 at columns 0..31 and rows 64..127 at columns 64..95
+// (one warp packs each 64-column half); by chunk (CHUNKS true), the 32 K rows
+// of chunk c at columns 32c..32c+15 (one warp packs each 32-column chunk
+// inside the columns it read).
+template <int D, int ELEM, bool CHUNKS = false>
 __device__ __forceinline__ void bwd_mma_ts_half(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, int h,
                                                 bool accumulate) {
   using C = BwdCfg<D, ELEM>;
@@ -165,7 +167,7 @@ __device__ __forceinline__ void bwd_mma_ts_half(uint32_t d_tmem, uint32_t a_tmem
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int kk = 4 * h + k;
-    const uint32_t a_col = kk * 8 + (kk >= 4 ? 32u : 0u);
+    const uint32_t a_col = CHUNKS ? (kk >> 1) * 32u + (kk & 1) * 8u : kk * 8 + (kk >= 4 ? 32u : 0u);
     mma_f16_ts(d_tmem, a_tmem + a_col, db + ((kk * 16 * C::SW) >> 4), C::IDESC_TS, (accumulate || k > 0) ? 1u : 0u);
   }
 }
@@ -249,7 +251,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int h = 0; h < 2; ++h) {
       mbar_init(b.s_full(h), 1);
-      mbar_init(b.p_full(h), 4);  // the four compute warps of column half h
+      mbar_init(b.p_full(h), 8);  // all eight compute warps, one chunk each
     }
     mbar_init(b.acc_full(), 1);
     mbar_init(b.mma_done(), 1);
@@ -329,8 +331,8 @@ __global__ void __launch_bounds__(320, 1)
           }
           FA_TRACE_EV(2, 60 + h, t);
           tc_fence_after();
-          bwd_mma_ts_half<D, ELEM>(tmem + C::COL_ACC0, tmem + C::COL_A, sDO, h, t > 0 || h > 0);  // dV += P^T_h dO_h
-          bwd_mma_ts_half<D, ELEM>(tmem + C::COL_ACC1, tmem + C::COL_B, sQ, h, t > 0 || h > 0);   // dK += dS^T_h Q_h
+          bwd_mma_ts_half<D, ELEM, true>(tmem + C::COL_ACC0, tmem + C::COL_A, sDO, h, t > 0 || h > 0);  // dV += P^T_h dO_h
+          bwd_mma_ts_half<D, ELEM, true>(tmem + C::COL_ACC1, tmem + C::COL_B, sQ, h, t > 0 || h > 0);   // dK += dS^T_h Q_h
           if (h == 1) tc_commit(b.empty(s));
           FA_TRACE_EV(2, 62 + h, t);
           if (next) {
@@ -354,59 +356,63 @@ __global__ void __launch_bounds__(320, 1)
       if (!wait_bounded(b.mma_done(), 0, &never, limit)) atomicOr(a.status, kStatusBwd);
     }
   } else {
-    // compute warps: thread = key row; warp w covers query columns 64(w/4)..+63
-    const int quarter = warp & 3, half = warp >> 2;
+    // compute warps: thread = key row; in column half h, warp w takes the
+    // 32-query chunk c = 2h + w/4 and packs its P^T and dS^T into the first
+    // 16 columns of that chunk, which only this warp reads
+    const int quarter = warp & 3, sub = warp >> 2;
     const int row = quarter * 32 + lane;
     const int key = 128 * j + row;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::COL_A, tP = tmem + lane_off + C::COL_B;
     const float* lse_h = a.lse + static_cast<size_t>(bh) * a.N;
     const float* dlt_h = a.delta + static_cast<size_t>(bh) * a.N;
-    // LSE and D of this warp's 64 query columns, fetched one query block
-    // ahead: lane l holds columns l and 32 + l in registers, and at the top of
+    // -LSE and -D of this warp's two chunks, fetched one query block ahead:
+    // lane l holds query l of each chunk in registers, and at the top of
     // each block the warp publishes them in its own shared-memory slot (only
     // __syncwarp orders it), from which every lane reads them as broadcasts.
     float pre_l[2], pre_d[2];
     auto prefetch = [&](int tt) {
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int qq = (i0 + tt) * 128 + 64 * half + 32 * u + lane;
+      for (int h = 0; h < 2; ++h) {
+        const int qq = (i0 + tt) * 128 + 32 * (2 * h + sub) + lane;
         const bool in_seq = tt < n_i && qq < a.N;
-        pre_l[u] = in_seq ? -(lse_h[qq] * 1.4426950408889634f) : 0.f;  // -LSE, log2 units
-        pre_d[u] = in_seq ? -dlt_h[qq] : 0.f;                           // -D
+        pre_l[h] = in_seq ? -(lse_h[qq] * 1.4426950408889634f) : 0.f;  // -LSE, log2 units
+        pre_d[h] = in_seq ? -dlt_h[qq] : 0.f;                           // -D
       }
     };
     prefetch(0);
     float* stage_l = lse_d_stage[warp][0];
     float* stage_d = lse_d_stage[warp][1];
+    const uint64_t sl2x2 = pack2(a.scale_log2, a.scale_log2);
     bool ok = true;
     FA_TRACE_DECL;
-    const bool tr = lane == 0 && quarter == 0;
+    const bool tr = lane == 0 && warp == 0;
     for (int t = 0; t < n_i && ok; ++t) {
       const int qb = (i0 + t) * 128;
       __syncwarp();  // every lane is done reading the previous block's values
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        stage_l[32 * u + lane] = pre_l[u];
-        stage_d[32 * u + lane] = pre_d[u];
+      for (int h = 0; h < 2; ++h) {
+        stage_l[32 * h + lane] = pre_l[h];
+        stage_d[32 * h + lane] = pre_d[h];
       }
       __syncwarp();
       prefetch(t + 1);  // in flight while this block computes
-      if (tr) FA_TRACE_EV(half, 70 + 10 * half, t);
-      ok = __all_sync(0xffffffffu, wait_bounded(b.s_full(half), t & 1, abort_flag, limit));
-      if (!ok) break;
-      tc_fence_after();
-      if (tr) FA_TRACE_EV(half, 71 + 10 * half, t);
 #pragma unroll 1
-      for (int c = 2 * half; c < 2 * half + 2; ++c) {
+      for (int h = 0; h < 2; ++h) {
+        if (tr) FA_TRACE_EV(h, 70 + 10 * h, t);
+        ok = __all_sync(0xffffffffu, wait_bounded(b.s_full(h), t & 1, abort_flag, limit));
+        if (!ok) break;
+        tc_fence_after();
+        if (tr) FA_TRACE_EV(h, 71 + 10 * h, t);
+        const int c = 2 * h + sub;
         ChunkIn in;
         tmem_ld32(tS + 32 * c, in.s);
         tmem_ld32(tP + 32 * c, in.dp);
         // -LSE (log2 units) and -D of the chunk's 32 queries (the same for every lane)
         const int q0 = qb + 32 * c;
         float nlse2[32], ndlt[32];
-        const float4* sl4 = reinterpret_cast<const float4*>(stage_l + 32 * (c - 2 * half));
-        const float4* sd4 = reinterpret_cast<const float4*>(stage_d + 32 * (c - 2 * half));
+        const float4* sl4 = reinterpret_cast<const float4*>(stage_l + 32 * h);
+        const float4* sd4 = reinterpret_cast<const float4*>(stage_d + 32 * h);
 #pragma unroll
         for (int v4 = 0; v4 < 8; ++v4) {
           const float4 l4 = sl4[v4], d4 = sd4[v4];
@@ -415,7 +421,7 @@ __global__ void __launch_bounds__(320, 1)
         }
         tmem_ld_wait(in.s);
         reg_tie(in.dp);
-        if (tr) FA_TRACE_EV(half, 72 + 10 * half + 2 * (c - 2 * half), t);
+        if (tr) FA_TRACE_EV(h, 72 + 10 * h, t);
         // Column e holds query q0 + e; it counts when that query exists and,
         // if causal, does not precede this key: lo <= e < hi.  Chunks with
         // every column valid (all but the tail and the diagonal) take the
@@ -424,7 +430,6 @@ __global__ void __launch_bounds__(320, 1)
         const int lo = a.causal ? min(max(key - q0, 0), 32) : 0;
         const uint32_t vmask = low_bits(hi) & ~low_bits(lo);
         uint32_t pp[16], pd[16];
-        const uint64_t sl2x2 = pack2(a.scale_log2, a.scale_log2);
         // two columns per packed instruction: p = 2^(s sl2 - LSE), ds = p (dp - D)
         auto chunk = [&](auto masked) {
 #pragma unroll
@@ -450,21 +455,20 @@ __global__ void __launch_bounds__(320, 1)
           chunk(std::false_type{});
         else
           chunk(std::true_type{});
-        tmem_st16(tS + 64 * half + 16 * (c - 2 * half), pp);
-        tmem_st16(tP + 64 * half + 16 * (c - 2 * half), pd);
-        if (tr) FA_TRACE_EV(half, 73 + 10 * half + 2 * (c - 2 * half), t);
+        tmem_st16(tS + 32 * c, pp);
+        tmem_st16(tP + 32 * c, pd);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b.p_full(h));
+        if (tr) FA_TRACE_EV(h, 76 + 10 * h, t);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(b.p_full(half));
-      if (tr) FA_TRACE_EV(half, 76 + 10 * half, t);
     }
     if (ok) ok = __all_sync(0xffffffffu, wait_bounded(b.acc_full(), 0, abort_flag, limit));
     if (ok) {
       tc_fence_after();
-      // warp half 0 stores dV, half 1 stores dK (this thread's key row)
-      if (half == 0)
+      // warps 0-3 store dV, warps 4-7 dK (this thread's key row)
+      if (sub == 0)
         bwd_store_acc<D, ELEM>(tmem + lane_off + C::COL_ACC0, a.dv, bh, a.N, key, 1.f);
       else
         bwd_store_acc<D, ELEM>(tmem + lane_off + C::COL_ACC1, a.dk, bh, a.N, key, a.scale);
