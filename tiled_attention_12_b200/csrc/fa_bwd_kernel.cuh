@@ -20,13 +20,17 @@
 //                      Computing dQ in its own pass (recomputing S and dP
 //                      once more) avoids fp32 atomics on dQ.
 //
-// Warps 0-7: compute (warp w: rows 32(w%4)..+31 of the 128-row tile, columns
-// 64(w/4)..+63 of the 128x128 score block); warp 8: TMA producer; warp 9:
-// tensor-memory allocation and the MMA-issuing thread.  Both kernels are
-// pipelined by column half: the scores of each 64-column half are issued as
-// their own N = 64 products with their own barrier, the half's four warps
-// hand P/dS back on another, and the MMA thread accumulates that half and
-// issues the next block's scores for it while the other half computes.
+// Warps 0-7: compute (warp w: rows 32(w%4)..+31 of the 128-row tile; in
+// column half h, the 32-column chunk 2h + w/4 of the 128x128 score block);
+// warp 8: TMA producer; warp 9: tensor-memory allocation and the
+// MMA-issuing thread.  Both kernels are pipelined by column half: the
+// scores of each 64-column half are issued as their own N = 64 products with
+// their own barrier, all eight warps turn that half into P/dS (each packing
+// its chunk inside the columns it read) and hand it back on another, and the
+// MMA thread accumulates that half and issues the next block's scores for it
+// while the warps compute the other half.  The per-column masks (sequence
+// end, causal diagonal) are bitmasks built once per chunk; chunks with every
+// column valid run without selects.
 // Tensor memory (dK/dV kernel): S^T [0,128), dP^T [128,256), dV [256,256+d),
 // dK [256+d,256+2d); (dQ kernel): S [0,128), dP [128,256), dQ [256,256+d).
 // Every wait is bounded as in the forward kernel.
@@ -154,12 +158,10 @@ __device__ __forceinline__ void bwd_mma_ss_half(uint32_t d_tmem, uint32_t a_smem
 
 // acc (+)= A_h B_h: A (128 x 128, 16-bit, packed) in tensor memory at
 // a_tmem, B a 128-row tile in shared memory read N-major (its rows are the K
-// index); only K rows 64h..64h+63.  Packed A layouts: by half (CHUNKS
-// false), K rows 0..63 at columns 0..31 and rows 64..127 at columns 64..95
-// (one warp packs each 64-column half); by chunk (CHUNKS true), the 32 K rows
-// of chunk c at columns 32c..32c+15 (one warp packs each 32-column chunk
+// index); only K rows 64h..64h+63.  The packed A keeps the 32 K rows of chunk
+// c at columns 32c..32c+15 (one compute warp packs each 32-column chunk
 // inside the columns it read).
-template <int D, int ELEM, bool CHUNKS = false>
+template <int D, int ELEM>
 __device__ __forceinline__ void bwd_mma_ts_half(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, int h,
                                                 bool accumulate) {
   using C = BwdCfg<D, ELEM>;
@@ -167,7 +169,7 @@ __device__ __forceinline__ void bwd_mma_ts_half(uint32_t d_tmem, uint32_t a_tmem
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int kk = 4 * h + k;
-    const uint32_t a_col = CHUNKS ? (kk >> 1) * 32u + (kk & 1) * 8u : kk * 8 + (kk >= 4 ? 32u : 0u);
+    const uint32_t a_col = (kk >> 1) * 32u + (kk & 1) * 8u;
     mma_f16_ts(d_tmem, a_tmem + a_col, db + ((kk * 16 * C::SW) >> 4), C::IDESC_TS, (accumulate || k > 0) ? 1u : 0u);
   }
 }
@@ -331,8 +333,8 @@ __global__ void __launch_bounds__(320, 1)
           }
           FA_TRACE_EV(2, 60 + h, t);
           tc_fence_after();
-          bwd_mma_ts_half<D, ELEM, true>(tmem + C::COL_ACC0, tmem + C::COL_A, sDO, h, t > 0 || h > 0);  // dV += P^T_h dO_h
-          bwd_mma_ts_half<D, ELEM, true>(tmem + C::COL_ACC1, tmem + C::COL_B, sQ, h, t > 0 || h > 0);   // dK += dS^T_h Q_h
+          bwd_mma_ts_half<D, ELEM>(tmem + C::COL_ACC0, tmem + C::COL_A, sDO, h, t > 0 || h > 0);  // dV += P^T_h dO_h
+          bwd_mma_ts_half<D, ELEM>(tmem + C::COL_ACC1, tmem + C::COL_B, sQ, h, t > 0 || h > 0);   // dK += dS^T_h Q_h
           if (h == 1) tc_commit(b.empty(s));
           FA_TRACE_EV(2, 62 + h, t);
           if (next) {
@@ -516,7 +518,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int h = 0; h < 2; ++h) {
       mbar_init(b.s_full(h), 1);
-      mbar_init(b.p_full(h), 4);  // the four compute warps of column half h
+      mbar_init(b.p_full(h), 8);  // all eight compute warps, one chunk each
     }
     mbar_init(b.acc_full(), 1);
     mbar_init(b.mma_done(), 1);
@@ -610,8 +612,10 @@ __global__ void __launch_bounds__(320, 1)
       if (!wait_bounded(b.mma_done(), 0, &never, limit)) atomicOr(a.status, kStatusBwd);
     }
   } else {
-    // compute warps: thread = query row; warp w covers key columns 64(w/4)..+63
-    const int quarter = warp & 3, half = warp >> 2;
+    // compute warps: thread = query row; in key half h, warp w takes the
+    // 32-key chunk c = 2h + w/4 and packs its dS into the first 16 columns of
+    // that chunk, which only this warp reads
+    const int quarter = warp & 3, sub = warp >> 2;
     const int row = quarter * 32 + lane;
     const int qrow = 128 * i + row;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -621,18 +625,25 @@ __global__ void __launch_bounds__(320, 1)
     const float dlt = row_ok ? a.delta[static_cast<size_t>(bh) * a.N + qrow] : 0.f;
     const uint64_t sl2x2 = pack2(a.scale_log2, a.scale_log2);
     const uint64_t nlse2x2 = pack2(-lse2, -lse2), ndltx2 = pack2(-dlt, -dlt);
+    // keys past the sequence end, or after the query when causal, are masked
+    const int limit_key = (a.causal && qrow < a.N - 1) ? qrow : a.N - 1;
     bool ok = true;
     for (int t = 0; t < n_j && ok; ++t) {
-      ok = __all_sync(0xffffffffu, wait_bounded(b.s_full(half), t & 1, abort_flag, limit));
-      if (!ok) break;
-      tc_fence_after();
       const int kb = 128 * t;
-      // keys past the sequence end, or after the query when causal, are masked
-      const int limit_key = (a.causal && qrow < a.N - 1) ? qrow : a.N - 1;
-      // dS of one 32-key chunk from its S and dP columns, packed in place
-      // (column e holds key kb + 32c + e: valid for e < hi; chunks with
-      // every column valid take the loop without selects)
-      auto chunk_ds = [&](const ChunkIn& in, int c) {
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        ok = __all_sync(0xffffffffu, wait_bounded(b.s_full(h), t & 1, abort_flag, limit));
+        if (!ok) break;
+        tc_fence_after();
+        const int c = 2 * h + sub;
+        ChunkIn in;
+        tmem_ld32(tS + 32 * c, in.s);
+        tmem_ld32(tP + 32 * c, in.dp);
+        tmem_ld_wait(in.s);
+        reg_tie(in.dp);
+        // dS of the chunk from its S and dP columns (column e holds key
+        // kb + 32c + e: valid for e < hi; chunks with every column valid take
+        // the loop without selects)
         const int hi = row_ok ? min(max(limit_key - kb - 32 * c + 1, 0), 32) : 0;
         const uint32_t vmask = low_bits(hi);
         uint32_t pd[16];
@@ -656,30 +667,17 @@ __global__ void __launch_bounds__(320, 1)
           body(std::false_type{});
         else
           body(std::true_type{});
-        tmem_st16(tS + 64 * half + 16 * (c - 2 * half), pd);
-      };
-      // both chunks' loads in flight together: one tensor-memory latency
-      ChunkIn in0, in1;
-      tmem_ld32(tS + 64 * half, in0.s);
-      tmem_ld32(tP + 64 * half, in0.dp);
-      tmem_ld32(tS + 64 * half + 32, in1.s);
-      tmem_ld32(tP + 64 * half + 32, in1.dp);
-      tmem_ld_wait(in0.s);
-      reg_tie(in0.dp);
-      reg_tie(in1.s);
-      reg_tie(in1.dp);
-      chunk_ds(in0, 2 * half);
-      chunk_ds(in1, 2 * half + 1);
-
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(b.p_full(half));
+        tmem_st16(tS + 32 * c, pd);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b.p_full(h));
+      }
     }
     if (ok) ok = __all_sync(0xffffffffu, wait_bounded(b.acc_full(), 0, abort_flag, limit));
     if (ok) {
       tc_fence_after();
-      if (half == 0) bwd_store_acc<D, ELEM>(tmem + lane_off + C::COL_ACC0, a.dq, bh, a.N, qrow, a.scale);
+      if (sub == 0) bwd_store_acc<D, ELEM>(tmem + lane_off + C::COL_ACC0, a.dq, bh, a.N, qrow, a.scale);
     } else {
       *abort_flag = 1;
       atomicOr(a.status, kStatusBwd);
