@@ -749,10 +749,19 @@ __device__ __forceinline__ void load_s_row(uint32_t t_s, uint32_t (&sr)[4][32]) 
 
 // Keys past limit_key (the sequence end, or the query itself when causal)
 // become -inf.  Only the last K/V tile of a row block can hold such keys.
+// The kept columns are 0..limit_key - kbase: one count per row, a bitmask
+// per 32-column chunk, and nothing to do when all 128 are kept.
 __device__ __forceinline__ void mask_row(uint32_t (&sr)[4][32], int kbase, int limit_key) {
+  const int kept = limit_key - kbase + 1;
+  if (kept >= 128) return;
 #pragma unroll
-  for (int c = 0; c < 128; ++c)
-    if (kbase + c > limit_key) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+  for (int ch = 0; ch < 4; ++ch) {
+    const int n = min(max(kept - 32 * ch, 0), 32);
+    const uint32_t keep = n >= 32 ? 0xffffffffu : (1u << n) - 1u;
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      sr[ch][e] = (keep >> e) & 1u ? sr[ch][e] : __float_as_uint(-INFINITY);
+  }
 }
 
 __device__ __forceinline__ float row_max(const uint32_t (&sr)[4][32]) {
