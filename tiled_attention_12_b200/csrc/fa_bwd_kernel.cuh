@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(320, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t tmem_holder;
   __shared__ int abort_storage;
-  // per compute warp: LSE (log2 units) and D of its 64 query columns
+  // per compute warp: -LSE (log2 units) and -D of the 32 queries of each of its two chunks
   __shared__ __align__(16) float lse_d_stage[8][2][64];
   volatile int* abort_flag = &abort_storage;
   const uint32_t raw = smem_u32(smem_raw);
