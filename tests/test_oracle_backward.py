@@ -56,6 +56,16 @@ def test_dv_closed_form_for_zero_q():
     assert np.max(np.abs(dv[0, 0] - np.sum(g[0, 0], axis=0) / n)) < 1e-12
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_single_key_closed_form(causal):
+    """N = 1: O = V, so dV = dO; P = 1 makes dS = P (dP - D) = dO.V - dO.V = 0,
+    so dQ = dK = 0 exactly, whatever Q, K and the scale."""
+    q, k, v, g = (_rand((2, 3, 1, 5), s) for s in (11, 12, 13, 14))
+    dq, dk, dv = attention_bwd_ref(q, k, v, g, 0.9, causal)
+    assert np.max(np.abs(dv - g)) < 1e-15
+    assert np.max(np.abs(dq)) < 1e-15 and np.max(np.abs(dk)) < 1e-15
+
+
 def test_gradient_identities():
     """Adding a constant to every score of a row leaves softmax unchanged, so
     each row of dS sums to zero and therefore sum_j dK_j = scale * dS^T Q
